@@ -1,0 +1,47 @@
+"""Plant a mistake in the oracle, on the CPU, and check that a pin catches it.
+
+Each case edits one line of a copy of oracle/mxfp8_oracle.c (an off-by-one
+scale exponent, ties to odd, a transposed weight index, a dropped bias, a
+wrong scale index, overflow to NaN instead of saturation, a lost sign), builds the copy and
+runs the pins against it; the pins must fail.  The real oracle is untouched.
+"""
+import os
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "mxfp8_oracle.c")
+
+MUTATIONS = {
+    "scale_exponent_off_by_one": ("e = (ex - 1) - 8;", "e = ex - 8;"),
+    "ties_to_odd": ("pick = (lo & 1) ? lo + 1 : lo;", "pick = (lo & 1) ? lo : lo + 1;"),
+    "weight_transposed": ("wq[n * K + k]", "wq[k * N + n]"),
+    "bias_dropped": ("acc += orc_f16_decode(bias[n]);", "acc += 0.0;"),
+    "scale_index_wrong": ("xs[r * nb + k / 32]", "xs[r * nb + k % nb]"),
+    "overflow_to_nan": ("if (a >= e4m3_mag[0x7E])\n        return sign | 0x7E;",
+                        "if (a >= e4m3_mag[0x7E])\n        return sign | 0x7F;"),
+    "sign_lost": ("return sign | (uint8_t)pick;", "return (uint8_t)pick;"),
+    "subnormal_scale_wrong": ("mag = ldexp((double)m, -9);", "mag = ldexp((double)m, -10);"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(name):
+    old, new = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation anchor not found: {old!r}"
+    mutated = src.replace(old, new)
+    with tempfile.TemporaryDirectory() as td:
+        c = os.path.join(td, "m.c")
+        so = os.path.join(td, "libm.so")
+        open(c, "w").write(mutated)
+        subprocess.run(["gcc", "-O1", "-std=c11", "-D_DEFAULT_SOURCE", "-fPIC", "-shared",
+                        "-fopenmp", "-ffp-contract=off", "-o", so, c, "-lm"], check=True)
+        env = dict(os.environ, ORACLE_LIB=so, OMP_NUM_THREADS="2")
+        r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                            os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                           cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+        assert r.returncode != 0, f"pins did not catch mutation {name}:\n{r.stdout[-2000:]}"
