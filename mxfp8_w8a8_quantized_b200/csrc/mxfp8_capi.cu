@@ -1,0 +1,204 @@
+/*
+ * mxfp8_capi.cu -- the C-ABI entry points declared in include/mxfp8.h:
+ * argument checks, then kernel launches on the caller's stream.
+ */
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "mxfp8.h"
+
+namespace mx {
+cudaError_t launch_quantize(const void *X, bool f32_in, int64_t M, int64_t K, int64_t ldx, uint8_t *Q, uint8_t *S,
+                            bool sf_tc, cudaStream_t stream);
+cudaError_t launch_gelu(const void *X, void *Y, int64_t n, cudaStream_t stream);
+int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void *Wq, const void *Ws, int64_t N,
+                const void *bias, void *Y, cudaStream_t stream, unsigned long long timeout_ns, cudaError_t *err);
+cudaError_t read_and_clear_status(unsigned int *out);
+} // namespace mx
+
+namespace {
+
+/* Bound for every pipeline wait inside the GEMM kernel. */
+constexpr unsigned long long kWaitLimitNs = 4000000000ull;
+
+/* Largest extents the kernels index with 32-bit tile arithmetic. */
+constexpr int64_t kMaxRows = (int64_t)1 << 30;
+constexpr int64_t kMaxK = (int64_t)1 << 20;
+
+bool aligned(const void *p, uintptr_t a)
+{
+    return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+size_t round_up(size_t v, size_t a)
+{
+    return (v + a - 1) / a * a;
+}
+
+mxfp8_status quantize_args(const void *X, int64_t M, int64_t K, int64_t ldx, const void *codes, const void *scales,
+                           int layout, size_t in_elem_bytes)
+{
+    if (!X || !codes || !scales)
+        return M == 0 ? MXFP8_OK : MXFP8_ERR_ARG;
+    if (layout != MXFP8_SF_ROWMAJOR && layout != MXFP8_SF_TCGEN05)
+        return MXFP8_ERR_ARG;
+    if (M < 0 || K <= 0 || ldx < K)
+        return MXFP8_ERR_ARG;
+    if (K % 32 != 0 || M > kMaxRows || K > kMaxK)
+        return MXFP8_ERR_SHAPE;
+    if (!aligned(X, 16) || (ldx * (int64_t)in_elem_bytes) % 16 != 0 || !aligned(codes, 8) || !aligned(scales, 4))
+        return MXFP8_ERR_ALIGN;
+    return MXFP8_OK;
+}
+
+mxfp8_status gemm_args(const void *A, const void *As, int64_t M, int64_t K, const void *Wq, const void *Ws,
+                       int64_t N, const void *bias, const void *Y)
+{
+    if (M < 0 || K <= 0 || N <= 0)
+        return MXFP8_ERR_ARG;
+    if (M == 0)
+        return MXFP8_OK;
+    if (!A || !As || !Wq || !Ws || !Y)
+        return MXFP8_ERR_ARG;
+    if (K % 128 != 0 || N % 8 != 0 || M > kMaxRows || N > kMaxRows || K > kMaxK)
+        return MXFP8_ERR_SHAPE;
+    if (!aligned(A, 16) || !aligned(As, 16) || !aligned(Wq, 16) || !aligned(Ws, 16) || !aligned(Y, 16) ||
+        (bias && !aligned(bias, 16)))
+        return MXFP8_ERR_ALIGN;
+    return MXFP8_OK;
+}
+
+mxfp8_status from_cuda(cudaError_t e)
+{
+    return e == cudaSuccess ? MXFP8_OK : MXFP8_ERR_CUDA;
+}
+
+} // namespace
+
+extern "C" {
+
+const char *mxfp8_status_str(mxfp8_status s)
+{
+    switch (s) {
+    case MXFP8_OK:
+        return "MXFP8_OK";
+    case MXFP8_ERR_ARG:
+        return "MXFP8_ERR_ARG: invalid argument (null pointer, bad layout or negative size)";
+    case MXFP8_ERR_ALIGN:
+        return "MXFP8_ERR_ALIGN: pointer or leading dimension not aligned";
+    case MXFP8_ERR_SHAPE:
+        return "MXFP8_ERR_SHAPE: unsupported shape (K % 32, K % 128 for the GEMM, N % 8, size limits)";
+    case MXFP8_ERR_CUDA:
+        return "MXFP8_ERR_CUDA: a CUDA call or kernel launch failed";
+    case MXFP8_ERR_TIMEOUT:
+        return "MXFP8_ERR_TIMEOUT: a kernel gave up a bounded pipeline wait";
+    }
+    return "MXFP8_ERR_UNKNOWN";
+}
+
+size_t mxfp8_scale_bytes(int64_t rows, int64_t K, int layout)
+{
+    if (rows < 0 || K <= 0 || K % 32 != 0)
+        return 0;
+    if (layout == MXFP8_SF_ROWMAJOR)
+        return (size_t)rows * (size_t)(K / 32);
+    if (layout == MXFP8_SF_TCGEN05)
+        return (size_t)((rows + 127) / 128) * (size_t)((K + 127) / 128) * 512u;
+    return 0;
+}
+
+mxfp8_status mxfp8_quantize(const void *X, int64_t M, int64_t K, int64_t ldx, void *codes, void *scales, int layout,
+                            mxfp8_stream_t stream)
+{
+    mxfp8_status st = quantize_args(X, M, K, ldx, codes, scales, layout, 2);
+    if (st != MXFP8_OK || M == 0)
+        return st;
+    return from_cuda(mx::launch_quantize(X, false, M, K, ldx, static_cast<uint8_t *>(codes),
+                                         static_cast<uint8_t *>(scales), layout == MXFP8_SF_TCGEN05,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mxfp8_status mxfp8_quantize_weight_f32(const float *W, int64_t N, int64_t K, void *Wq, void *Wscale, int layout,
+                                       mxfp8_stream_t stream)
+{
+    mxfp8_status st = quantize_args(W, N, K, K, Wq, Wscale, layout, 4);
+    if (st != MXFP8_OK || N == 0)
+        return st;
+    return from_cuda(mx::launch_quantize(W, true, N, K, K, static_cast<uint8_t *>(Wq), static_cast<uint8_t *>(Wscale),
+                                         layout == MXFP8_SF_TCGEN05, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t mxfp8_linear_workspace_bytes(int64_t M, int64_t K)
+{
+    if (M < 0 || K <= 0 || K % 32 != 0)
+        return 0;
+    return round_up((size_t)M * (size_t)K, 256) + mxfp8_scale_bytes(M, K, MXFP8_SF_TCGEN05);
+}
+
+mxfp8_status mxfp8_gemm_prequant(const void *Xq, const void *Xscale, int64_t M, int64_t K, const void *Wq,
+                                 const void *Wscale, int64_t N, const void *bias, void *Y, mxfp8_stream_t stream)
+{
+    mxfp8_status st = gemm_args(Xq, Xscale, M, K, Wq, Wscale, N, bias, Y);
+    if (st != MXFP8_OK || M == 0)
+        return st;
+    cudaError_t e;
+    int r = mx::launch_gemm(Xq, Xscale, M, K, Wq, Wscale, N, bias, Y, reinterpret_cast<cudaStream_t>(stream),
+                            kWaitLimitNs, &e);
+    if (r == 1)
+        return MXFP8_ERR_CUDA; /* tensor map could not be encoded */
+    return r == 0 ? MXFP8_OK : from_cuda(e);
+}
+
+mxfp8_status mxfp8_linear(const void *X, int64_t M, int64_t K, const void *Wq, const void *Wscale, int64_t N,
+                          const void *bias, void *Y, void *workspace, size_t ws_bytes, mxfp8_stream_t stream)
+{
+    if (M < 0 || K <= 0 || N <= 0)
+        return MXFP8_ERR_ARG;
+    if (M == 0)
+        return MXFP8_OK;
+    if (!X || !workspace)
+        return MXFP8_ERR_ARG;
+    if (K % 128 != 0)
+        return MXFP8_ERR_SHAPE;
+    if (!aligned(workspace, 256) || !aligned(X, 16))
+        return MXFP8_ERR_ALIGN;
+    if (ws_bytes < mxfp8_linear_workspace_bytes(M, K))
+        return MXFP8_ERR_ARG;
+    uint8_t *codes = static_cast<uint8_t *>(workspace);
+    uint8_t *scales = codes + round_up((size_t)M * (size_t)K, 256);
+    mxfp8_status st = gemm_args(codes, scales, M, K, Wq, Wscale, N, bias, Y);
+    if (st != MXFP8_OK)
+        return st;
+    st = mxfp8_quantize(X, M, K, K, codes, scales, MXFP8_SF_TCGEN05, stream);
+    if (st != MXFP8_OK)
+        return st;
+    return mxfp8_gemm_prequant(codes, scales, M, K, Wq, Wscale, N, bias, Y, stream);
+}
+
+mxfp8_status mxfp8_gelu_tanh_bf16(const void *X, void *Y, int64_t n, mxfp8_stream_t stream)
+{
+    if (n < 0)
+        return MXFP8_ERR_ARG;
+    if (n == 0)
+        return MXFP8_OK;
+    if (!X || !Y)
+        return MXFP8_ERR_ARG;
+    if (n % 8 != 0)
+        return MXFP8_ERR_SHAPE;
+    if (!aligned(X, 16) || !aligned(Y, 16))
+        return MXFP8_ERR_ALIGN;
+    return from_cuda(mx::launch_gelu(X, Y, n, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mxfp8_status mxfp8_device_status(mxfp8_stream_t stream)
+{
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return MXFP8_ERR_CUDA;
+    unsigned int word = 0;
+    if (mx::read_and_clear_status(&word) != cudaSuccess)
+        return MXFP8_ERR_CUDA;
+    return word ? MXFP8_ERR_TIMEOUT : MXFP8_OK;
+}
+
+} // extern "C"

@@ -1,0 +1,587 @@
+/*
+ * mxfp8_gemm.cu -- block-scaled MXFP8 GEMM with F16-bias / BF16 epilogue on
+ * the sm_100a tensor cores (tcgen05).
+ *
+ *   Y[m, n] = BF16_RNE( sum_b 2^(sx[m,b] + sw[n,b]) sum_{j<32} x[m,32b+j] w[n,32b+j]
+ *                       + F32(bias[n]) )
+ *
+ * (model card "Wan2.2-I2V-A14B-Lightning . MXFP8 (AutoRound OptRTN)":
+ * "Performance Profile" -- "linear (MXFP8 W8A8)" is the layer's GEMM;
+ * "Coverage per transformer" -- E4M3 codes, per-32 E8M0 scales, F16 biases.)
+ *
+ * Two variants of one persistent, warp-specialized kernel:
+ *
+ *  PAIR (default): a cluster of two CTAs on two SMs computes 256 x 256 output
+ *   tiles with tcgen05.mma.cta_group::2 (M = 256).  Each CTA stages its own
+ *   128 rows of A, its own half (128 rows) of B, the scale atom of its A rows
+ *   and both scale atoms of B, so per SM the tensor core is fed 64 bytes per
+ *   clock instead of the 96 a single-SM 128 x 256 tile needs -- the L2-to-SM
+ *   fabric, not the tensor core, limits the single-SM form on B200.  Loads
+ *   use TMA without multicast; their completion is signalled to the leader
+ *   CTA's barrier (cta_group::2 form), and the leader's single MMA thread
+ *   issues the MMAs for the pair.
+ *  SINGLE: one CTA per SM, 128 x 256 tiles, tcgen05.mma.cta_group::1.
+ *
+ * Roles (320 threads per CTA):
+ *   warp 0       TMA producer: per 128-wide K step, A and B tiles (tiled TMA,
+ *                128-byte swizzle) and their scale atoms (512 B per 128
+ *                rows, 3-D tiled TMA) into a multi-stage smem ring guarded
+ *                by mbarriers.
+ *   warp 1       allocates 512 TMEM columns; one thread (the leader CTA's in
+ *                PAIR) copies the stage's scales to TMEM (tcgen05.cp
+ *                32x128b.warpx4) and issues four tcgen05.mma
+ *                kind::mxf8f6f4.block_scale of K = 32, the scale byte of each
+ *                K step picked by the instruction descriptor's scale-factor
+ *                ID; tcgen05.commit frees the stage (in both CTAs) and, after
+ *                the tile, signals the epilogues.
+ *   warps 2..9   epilogue: each warp owns one 32-lane TMEM sub-partition and
+ *                half the columns; it drains its 32 x 128 FP32 block in one
+ *                tcgen05.ld, releases the accumulator to the MMA thread at
+ *                once, then adds the bias, rounds to BF16 and stores (rows
+ *                >= M and columns >= N masked) while the next tile's MMAs run.
+ * Scale columns in TMEM are per stage, so a scale copy never overwrites
+ * scales an earlier, still running MMA reads.  Every wait is bounded: on
+ * timeout the kernel records MXFP8_ERR_TIMEOUT in a device status word,
+ * drains its own MMAs, frees TMEM and returns.
+ */
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <cstdlib>
+
+#include "ptx.cuh"
+
+namespace mx {
+
+constexpr int BK = 128; /* bytes = E4M3 elements per K step */
+constexpr int EPI_WARPS = 8;
+constexpr int GEMM_THREADS = (2 + EPI_WARPS) * 32;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0; /* 256 FP32 columns */
+constexpr int RASTER_GROUP = 8; /* M tiles walked together for L2 reuse */
+constexpr uint32_t ST_TIMEOUT = 1u;
+
+template <bool PAIR>
+struct Cfg {
+    static constexpr int STAGES = PAIR ? 6 : 4;
+    static constexpr int TILE_M = PAIR ? 256 : 128; /* output rows per tile */
+    static constexpr int TILE_N = 256;
+    static constexpr uint32_t A_ROWS = 128;                 /* A rows staged per CTA */
+    static constexpr uint32_t B_ROWS = PAIR ? 128 : 256;    /* B rows staged per CTA */
+    static constexpr uint32_t A_BYTES = A_ROWS * BK;
+    static constexpr uint32_t B_BYTES = B_ROWS * BK;
+    static constexpr uint32_t SFA_BYTES = 512;              /* one atom: this CTA's 128 A rows */
+    static constexpr uint32_t SFB_BYTES = 1024;             /* two atoms: all 256 B rows */
+    static constexpr uint32_t STAGE_TX = (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) * (PAIR ? 2u : 1u);
+    static constexpr uint32_t SFA_COL = 256;                /* + 4 per stage */
+    static constexpr uint32_t SFB_COL = 256 + 4 * STAGES;   /* + 8 per stage */
+    static_assert(SFB_COL + 8 * STAGES <= TMEM_COLS, "TMEM budget");
+    static constexpr uint32_t OFF_A = 0;
+    static constexpr uint32_t OFF_B = OFF_A + STAGES * A_BYTES;
+    static constexpr uint32_t OFF_SFA = OFF_B + STAGES * B_BYTES;
+    static constexpr uint32_t OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
+    static constexpr uint32_t OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
+    static constexpr uint32_t NUM_BARS = 2 * STAGES + 3; /* full[], empty[], tmem_full, tmem_empty, drain */
+    static constexpr uint32_t OFF_TMEMPTR = OFF_BAR + NUM_BARS * 8;
+    static constexpr uint32_t OFF_ABORT = OFF_TMEMPTR + 4;
+    static constexpr uint32_t SMEM_USED = OFF_TMEMPTR + 16;
+    static constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024; /* slack to align the base to 1 KiB */
+    static constexpr uint32_t TEMPTY_ARRIVALS = EPI_WARPS * (PAIR ? 2u : 1u);
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+__device__ unsigned int g_mx_status = 0;
+
+struct GemmParams {
+    const __half *bias;   /* [N] or null */
+    __nv_bfloat16 *Y;     /* [M, N] */
+    int M, N, K;
+    int num_m, num_n;     /* output tiles */
+    unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int &mb, int &nb)
+{
+    const int per_group = RASTER_GROUP * num_n;
+    const int g = t / per_group;
+    const int first = g * RASTER_GROUP;
+    const int gm = min(RASTER_GROUP, num_m - first);
+    const int r = t - g * per_group;
+    mb = first + r % gm;
+    nb = r / gm;
+}
+
+/*
+ * Bounded wait: true when the phase of parity `parity` has completed.  On
+ * timeout it records ST_TIMEOUT in the device status word and raises the
+ * CTA's abort flag, so the other roles stop waiting too.
+ */
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, unsigned long long limit_ns,
+                                             volatile uint32_t *abort_flag)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 256; ++i)
+            if (mbar_try_wait(bar, parity))
+                return true;
+        if (*abort_flag)
+            return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            *abort_flag = 1u;
+            atomicOr(&g_mx_status, ST_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+template <bool PAIR>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                      const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
+                      const GemmParams p)
+{
+    using C = Cfg<PAIR>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    uint8_t *smem = smem_raw + (sbase - raw);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u; /* 0 = leader */
+    const int tile0 = PAIR ? (int)cluster_id_x() : (int)blockIdx.x;
+    const int tstep = PAIR ? (int)nclusters_x() : (int)gridDim.x;
+
+    const uint32_t bar_full = sbase + C::OFF_BAR;          /* + 8 s */
+    const uint32_t bar_empty = bar_full + C::STAGES * 8;   /* + 8 s */
+    const uint32_t bar_tfull = bar_empty + C::STAGES * 8;
+    const uint32_t bar_tempty = bar_tfull + 8;
+    const uint32_t bar_drain = bar_tempty + 8;
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + C::OFF_TMEMPTR);
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_ABORT);
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0u;
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        mbar_init(bar_tfull, 1);
+        mbar_init(bar_tempty, C::TEMPTY_ARRIVALS);
+        mbar_init(bar_drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        if constexpr (PAIR) {
+            tmem_alloc_pair(smem_u32(tmem_ptr), TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(tmem_ptr), TMEM_COLS);
+            tmem_relinquish();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if constexpr (PAIR)
+        cluster_sync_all(); /* peer barriers initialised before any remote signal */
+    tc_fence_after();
+    const uint32_t tmem = *tmem_ptr;
+
+    const int KB = p.K / BK;
+    const int num_tiles = p.num_m * p.num_n;
+    const unsigned long long lim = p.timeout_ns;
+
+    if (warp == 0) {
+        /* ------------------------------------------------ TMA producer */
+        if (lane == 0) {
+            prefetch_tmap(&tmap_a);
+            prefetch_tmap(&tmap_b);
+            prefetch_tmap(&tmap_sfa);
+            prefetch_tmap(&tmap_sfb);
+            uint32_t it = 0;
+            bool ok = true;
+            for (int t = tile0; ok && t < num_tiles; t += tstep) {
+                int mb, nb;
+                tile_coords(t, p.num_m, p.num_n, mb, nb);
+                const int rowA = mb * C::TILE_M + (int)(rank * 128u);
+                const int rowB = nb * C::TILE_N + (int)(rank * C::B_ROWS);
+                const int rbA = rowA / 128;
+                const int rbB = nb * 2;
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const uint32_t s = it % C::STAGES, ph = (it / C::STAGES) & 1u;
+                    if (!wait_bounded(bar_empty + 8 * s, ph ^ 1u, lim, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t full = bar_full + 8 * s;
+                    if (rank == 0)
+                        mbar_arrive_expect_tx(full, C::STAGE_TX);
+                    const uint32_t dA = sbase + C::OFF_A + s * C::A_BYTES;
+                    const uint32_t dB = sbase + C::OFF_B + s * C::B_BYTES;
+                    const uint32_t dSA = sbase + C::OFF_SFA + s * C::SFA_BYTES;
+                    const uint32_t dSB = sbase + C::OFF_SFB + s * C::SFB_BYTES;
+                    if constexpr (PAIR) {
+                        const uint32_t lead = mapa_shared(full, 0u);
+                        tma_load_2d_pair(dA, &tmap_a, kb * BK, rowA, lead);
+                        tma_load_2d_pair(dB, &tmap_b, kb * BK, rowB, lead);
+                        tma_load_3d_pair(dSA, &tmap_sfa, 0, kb, rbA, lead);
+                        tma_load_3d_pair(dSB, &tmap_sfb, 0, kb, rbB, lead);
+                    } else {
+                        tma_load_2d(dA, &tmap_a, kb * BK, rowA, full);
+                        tma_load_2d(dB, &tmap_b, kb * BK, rowB, full);
+                        tma_load_3d(dSA, &tmap_sfa, 0, kb, rbA, full);
+                        tma_load_3d(dSB, &tmap_sfb, 0, kb, rbB, full);
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        /* ------------------------------------------------ MMA issuer */
+        if (lane == 0 && rank == 0) {
+            const uint32_t idesc = idesc_mxf8_e4m3(C::TILE_M, C::TILE_N);
+            uint32_t it = 0, tl = 0;
+            bool ok = true, any = false;
+            for (int t = tile0; ok && t < num_tiles; t += tstep, ++tl) {
+                if (!wait_bounded(bar_tempty, (tl & 1u) ^ 1u, lim, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const uint32_t s = it % C::STAGES, ph = (it / C::STAGES) & 1u;
+                    if (!wait_bounded(bar_full + 8 * s, ph, lim, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t tsfa = tmem + C::SFA_COL + 4 * s;
+                    const uint32_t tsfb = tmem + C::SFB_COL + 8 * s;
+                    const uint32_t sfa_s = sbase + C::OFF_SFA + s * C::SFA_BYTES;
+                    const uint32_t sfb_s = sbase + C::OFF_SFB + s * C::SFB_BYTES;
+                    const uint64_t adesc = desc_kmajor_sw128(sbase + C::OFF_A + s * C::A_BYTES);
+                    const uint64_t bdesc = desc_kmajor_sw128(sbase + C::OFF_B + s * C::B_BYTES);
+                    if constexpr (PAIR) {
+                        tc_cp_32x128b_warpx4_pair(tsfa, desc_sf_32x16(sfa_s));
+                        tc_cp_32x128b_warpx4_pair(tsfb, desc_sf_32x16(sfb_s));
+                        tc_cp_32x128b_warpx4_pair(tsfb + 4, desc_sf_32x16(sfb_s + 512u));
+#pragma unroll
+                        for (int k = 0; k < BK / 32; ++k)
+                            tc_mma_mxf8_pair(tmem + ACC_COL, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k),
+                                             idesc_with_sf_id(idesc, (uint32_t)k), tsfa, tsfb, (kb | k) != 0);
+                        tc_commit_pair(bar_empty + 8 * s, (uint16_t)0x3);
+                    } else {
+                        tc_cp_32x128b_warpx4(tsfa, desc_sf_32x16(sfa_s));
+                        tc_cp_32x128b_warpx4(tsfb, desc_sf_32x16(sfb_s));
+                        tc_cp_32x128b_warpx4(tsfb + 4, desc_sf_32x16(sfb_s + 512u));
+#pragma unroll
+                        for (int k = 0; k < BK / 32; ++k)
+                            tc_mma_mxf8(tmem + ACC_COL, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k),
+                                        idesc_with_sf_id(idesc, (uint32_t)k), tsfa, tsfb, (kb | k) != 0);
+                        tc_commit(bar_empty + 8 * s);
+                    }
+                    any = true;
+                }
+                if (!ok)
+                    break;
+                if constexpr (PAIR)
+                    tc_commit_pair(bar_tfull, (uint16_t)0x3);
+                else
+                    tc_commit(bar_tfull);
+            }
+            if (ok && tl > 0) {
+                /* every epilogue (the peer's included) has released the last
+                 * accumulator, so no remote arrival is still in flight */
+                (void)wait_bounded(bar_tempty, (tl & 1u) ^ 1u, lim, abort_flag);
+            }
+            if (!ok && any) {
+                /* wait for this thread's MMAs and copies before TMEM is freed */
+                volatile uint32_t own = 0u;
+                if constexpr (PAIR)
+                    tc_commit_pair(bar_drain, (uint16_t)0x1);
+                else
+                    tc_commit(bar_drain);
+                (void)wait_bounded(bar_drain, 0u, lim, &own);
+            }
+        }
+    } else {
+        /* ------------------------------------------------ epilogue */
+        const int q = warp & 3;            /* TMEM sub-partition this warp may read */
+        const int h = (warp - 2) >> 2;     /* column half of the 256-wide tile */
+        const uint32_t tempty_lead = PAIR ? mapa_shared(bar_tempty, 0u) : bar_tempty;
+        uint32_t tl = 0;
+        for (int t = tile0; t < num_tiles; t += tstep, ++tl) {
+            int mb, nb;
+            tile_coords(t, p.num_m, p.num_n, mb, nb);
+            /* every lane polls; the vote keeps the warp converged for the
+             * .sync.aligned TMEM load and makes the outcome warp-uniform */
+            const bool got = wait_bounded(bar_tfull, tl & 1u, lim, abort_flag);
+            if (!__all_sync(0xFFFFFFFFu, got))
+                break;
+            tc_fence_after();
+            uint32_t acc[128];
+            tmem_ld_32x32b_x128_sync(tmem + ((uint32_t)(32 * q) << 16) + ACC_COL + (uint32_t)(h * 128), acc);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if constexpr (PAIR)
+                    mbar_arrive_cluster(tempty_lead);
+                else
+                    mbar_arrive(bar_tempty);
+            }
+
+            const int row = mb * C::TILE_M + (int)(rank * 128u) + 32 * q + lane;
+            const int col0 = nb * C::TILE_N + h * 128;
+            if (row < p.M) {
+                __nv_bfloat16 *yrow = p.Y + (size_t)row * p.N;
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const int col = col0 + 8 * c;
+                    if (col < p.N) {
+                        float b[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                        if (p.bias) {
+                            const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(p.bias + col));
+                            const __half2 *bh = reinterpret_cast<const __half2 *>(&bv);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const float2 f2 = __half22float2(bh[j]);
+                                b[2 * j] = f2.x;
+                                b[2 * j + 1] = f2.y;
+                            }
+                        }
+                        uint32_t o[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(acc[8 * c + 2 * j]) + b[2 * j],
+                                                                     __uint_as_float(acc[8 * c + 2 * j + 1]) +
+                                                                         b[2 * j + 1]);
+                            o[j] = *reinterpret_cast<uint32_t *>(&v);
+                        }
+                        *reinterpret_cast<uint4 *>(yrow + col) = make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if constexpr (PAIR)
+        cluster_sync_all(); /* neither CTA leaves while the pair may still touch it */
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        if constexpr (PAIR)
+            tmem_dealloc_pair(tmem, TMEM_COLS);
+        else
+            tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+/* ------------------------------------------------------------ host side */
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                    const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled get_encode_fn()
+{
+    static PFN_encodeTiled fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_encodeTiled>(p);
+    }
+    return fn;
+}
+
+/* K-major E4M3 operand [rows, K]: box 128 (K bytes) x box_rows, 128-byte swizzle. */
+static bool make_operand_map(CUtensorMap *m, const void *base, int64_t rows, int64_t K, uint32_t box_rows)
+{
+    PFN_encodeTiled enc = get_encode_fn();
+    if (!enc)
+        return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K};
+    cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+/* Scale array in the tensor-core layout viewed as [row blocks][K/128][128 u32]
+ * (one 512-byte atom per (row block, K step)); box = `atoms` consecutive row
+ * blocks of one K step.  Row blocks past the end read as zero. */
+static bool make_scale_map(CUtensorMap *m, const void *base, int64_t rows, int64_t K, uint32_t atoms)
+{
+    PFN_encodeTiled enc = get_encode_fn();
+    if (!enc)
+        return false;
+    const int64_t kg = K / 128, rb = (rows + 127) / 128;
+    cuuint64_t dims[3] = {128, (cuuint64_t)kg, (cuuint64_t)rb};
+    cuuint64_t strides[2] = {512, (cuuint64_t)(kg * 512)};
+    cuuint32_t box[3] = {128, 1, atoms};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct DevInfo {
+    bool init = false;
+    int sms = 148;
+    int max_pair_clusters = 0; /* 0: pairs unavailable */
+    bool attr_single = false, attr_pair = false;
+};
+static DevInfo g_dev[64];
+
+static DevInfo *dev_info()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return nullptr;
+    DevInfo &d = g_dev[dev];
+    if (!d.init) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+            d.sms = v;
+        d.init = true;
+    }
+    return &d;
+}
+
+template <bool PAIR>
+static cudaError_t launch_variant(const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorMap &msa,
+                                  const CUtensorMap &msb, const GemmParams &p, int grid, cudaStream_t stream)
+{
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(GEMM_THREADS);
+    cfg.dynamicSmemBytes = Cfg<PAIR>::SMEM_BYTES;
+    cfg.stream = stream;
+    if (PAIR) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, mxfp8_gemm_kernel<PAIR>, ma, mb, msa, msb, p);
+}
+
+/* Whether the CTA-pair variant is used: on unless MXFP8_GEMM_PAIR=0. */
+static bool pair_enabled()
+{
+    static int v = -1;
+    if (v < 0) {
+        const char *e = getenv("MXFP8_GEMM_PAIR");
+        v = (e && e[0] == '0') ? 0 : 1;
+    }
+    return v == 1;
+}
+
+/* 0 ok, 1 tensor-map failure, 2 CUDA error (in *err). */
+int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void *Wq, const void *Ws, int64_t N,
+                const void *bias, void *Y, cudaStream_t stream, unsigned long long timeout_ns, cudaError_t *err)
+{
+    *err = cudaSuccess;
+    if (M == 0)
+        return 0;
+    DevInfo *d = dev_info();
+    if (!d) {
+        *err = cudaErrorInvalidDevice;
+        return 2;
+    }
+    cudaError_t e;
+    bool pair = pair_enabled();
+    if (pair && !d->attr_pair) {
+        e = cudaFuncSetAttribute(mxfp8_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)Cfg<true>::SMEM_BYTES);
+        if (e == cudaSuccess) {
+            cudaLaunchConfig_t cfg = {};
+            cudaLaunchAttribute attr[1];
+            cfg.gridDim = dim3(2 * (unsigned)d->sms);
+            cfg.blockDim = dim3(GEMM_THREADS);
+            cfg.dynamicSmemBytes = Cfg<true>::SMEM_BYTES;
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, mxfp8_gemm_kernel<true>, &cfg) == cudaSuccess)
+                d->max_pair_clusters = n;
+            else
+                cudaGetLastError(); /* clear; fall back to single CTAs */
+        } else {
+            cudaGetLastError();
+        }
+        d->attr_pair = true;
+    }
+    if (pair && d->max_pair_clusters <= 0)
+        pair = false;
+    if (!pair && !d->attr_single) {
+        e = cudaFuncSetAttribute(mxfp8_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)Cfg<false>::SMEM_BYTES);
+        if (e != cudaSuccess) {
+            *err = e;
+            return 2;
+        }
+        d->attr_single = true;
+    }
+
+    const uint32_t b_rows = pair ? Cfg<true>::B_ROWS : Cfg<false>::B_ROWS;
+    CUtensorMap ma, mb, msa, msb;
+    if (!make_operand_map(&ma, Xq, M, K, 128) || !make_operand_map(&mb, Wq, N, K, b_rows) ||
+        !make_scale_map(&msa, Xs, M, K, 1) || !make_scale_map(&msb, Ws, N, K, 2))
+        return 1;
+    GemmParams p;
+    p.bias = static_cast<const __half *>(bias);
+    p.Y = static_cast<__nv_bfloat16 *>(Y);
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    const int tile_m = pair ? Cfg<true>::TILE_M : Cfg<false>::TILE_M;
+    p.num_m = (int)((M + tile_m - 1) / tile_m);
+    p.num_n = (int)((N + 255) / 256);
+    p.timeout_ns = timeout_ns;
+    const int tiles = p.num_m * p.num_n;
+    if (pair) {
+        int clusters = d->max_pair_clusters;
+        if (clusters > tiles)
+            clusters = tiles;
+        e = launch_variant<true>(ma, mb, msa, msb, p, 2 * clusters, stream);
+    } else {
+        int grid = d->sms;
+        if (grid > tiles)
+            grid = tiles;
+        e = launch_variant<false>(ma, mb, msa, msb, p, grid, stream);
+    }
+    if (e != cudaSuccess) {
+        *err = e;
+        return 2;
+    }
+    return 0;
+}
+
+/* Reads and clears the status word of the current device (synchronous). */
+cudaError_t read_and_clear_status(unsigned int *out)
+{
+    unsigned int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_mx_status, sizeof(unsigned int));
+    if (e != cudaSuccess)
+        return e;
+    return cudaMemcpyToSymbol(g_mx_status, &zero, sizeof(unsigned int));
+}
+
+} // namespace mx

@@ -1,0 +1,154 @@
+"""Thin ctypes binding over libmxfp8.so (C-ABI in include/mxfp8.h).
+
+Argument marshalling only: tensors are passed as device pointers together
+with the current CUDA stream, outputs are allocated with PyTorch.  Every step
+of the layer runs in the library's kernels; there is no CPU or library
+fallback, and importing this module raises if the library is missing.
+"""
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmxfp8.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m mxfp8_w8a8_quantized_b200.build` "
+        "(there is no fallback implementation)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+
+_lib.mxfp8_status_str.argtypes = [ctypes.c_int]
+_lib.mxfp8_status_str.restype = ctypes.c_char_p
+_lib.mxfp8_scale_bytes.argtypes = [_I64, _I64, ctypes.c_int]
+_lib.mxfp8_scale_bytes.restype = _SZ
+_lib.mxfp8_quantize.argtypes = [_P, _I64, _I64, _I64, _P, _P, ctypes.c_int, _P]
+_lib.mxfp8_quantize.restype = ctypes.c_int
+_lib.mxfp8_quantize_weight_f32.argtypes = [_P, _I64, _I64, _P, _P, ctypes.c_int, _P]
+_lib.mxfp8_quantize_weight_f32.restype = ctypes.c_int
+_lib.mxfp8_linear_workspace_bytes.argtypes = [_I64, _I64]
+_lib.mxfp8_linear_workspace_bytes.restype = _SZ
+_lib.mxfp8_linear.argtypes = [_P, _I64, _I64, _P, _P, _I64, _P, _P, _P, _SZ, _P]
+_lib.mxfp8_linear.restype = ctypes.c_int
+_lib.mxfp8_gemm_prequant.argtypes = [_P, _P, _I64, _I64, _P, _P, _I64, _P, _P, _P]
+_lib.mxfp8_gemm_prequant.restype = ctypes.c_int
+_lib.mxfp8_gelu_tanh_bf16.argtypes = [_P, _P, _I64, _P]
+_lib.mxfp8_gelu_tanh_bf16.restype = ctypes.c_int
+_lib.mxfp8_device_status.argtypes = [_P]
+_lib.mxfp8_device_status.restype = ctypes.c_int
+
+SF_ROWMAJOR = 0
+SF_TCGEN05 = 1
+
+EXPORTS = ("mxfp8_status_str", "mxfp8_scale_bytes", "mxfp8_quantize", "mxfp8_quantize_weight_f32",
+           "mxfp8_linear_workspace_bytes", "mxfp8_linear", "mxfp8_gemm_prequant",
+           "mxfp8_gelu_tanh_bf16", "mxfp8_device_status")
+
+
+class MXFP8Error(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {_lib.mxfp8_status_str(status).decode()}")
+
+
+def _check(status, where):
+    if status != 0:
+        raise MXFP8Error(status, where)
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _cuda(t, name, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def scale_bytes(rows: int, K: int, layout: int = SF_TCGEN05) -> int:
+    return int(_lib.mxfp8_scale_bytes(rows, K, layout))
+
+
+def linear_workspace_bytes(M: int, K: int) -> int:
+    return int(_lib.mxfp8_linear_workspace_bytes(M, K))
+
+
+def quantize(x: torch.Tensor, layout: int = SF_TCGEN05, codes=None, scales=None):
+    """BF16 [M, K] -> (E4M3 codes uint8 [M, K], E8M0 scales uint8 [bytes])."""
+    _cuda(x, "x", torch.bfloat16)
+    M, K = x.shape
+    if codes is None:
+        codes = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(max(scale_bytes(M, K, layout), 1), dtype=torch.uint8, device=x.device)
+    _check(_lib.mxfp8_quantize(_ptr(x), M, K, K, _ptr(codes), _ptr(scales), layout, _stream()),
+           "mxfp8_quantize")
+    return codes, scales
+
+
+def quantize_weight(w: torch.Tensor, layout: int = SF_TCGEN05):
+    """FP32 [N, K] -> (E4M3 codes uint8 [N, K], E8M0 scales uint8 [bytes])."""
+    _cuda(w, "w", torch.float32)
+    N, K = w.shape
+    codes = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    scales = torch.empty(max(scale_bytes(N, K, layout), 1), dtype=torch.uint8, device=w.device)
+    _check(_lib.mxfp8_quantize_weight_f32(_ptr(w), N, K, _ptr(codes), _ptr(scales), layout, _stream()),
+           "mxfp8_quantize_weight_f32")
+    return codes, scales
+
+
+def linear(x: torch.Tensor, wq: torch.Tensor, wscale: torch.Tensor, bias=None, out=None, workspace=None):
+    """Y = BF16(MXFP8(x) . MXFP8(W)^T + bias): x BF16 [M, K], wq [N, K], bias F16 [N]."""
+    _cuda(x, "x", torch.bfloat16)
+    _cuda(wq, "wq", torch.uint8)
+    _cuda(wscale, "wscale", torch.uint8)
+    M, K = x.shape
+    N = wq.shape[0]
+    if bias is not None:
+        _cuda(bias, "bias", torch.float16)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    ws = linear_workspace_bytes(M, K)
+    if workspace is None:
+        workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=x.device)
+    _check(_lib.mxfp8_linear(_ptr(x), M, K, _ptr(wq), _ptr(wscale), N, _ptr(bias), _ptr(out),
+                             _ptr(workspace), workspace.numel(), _stream()), "mxfp8_linear")
+    return out
+
+
+def gemm_prequant(xq, xscale, wq, wscale, bias=None, out=None):
+    """Y from operands already quantized (tensor-core scale layout)."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    _check(_lib.mxfp8_gemm_prequant(_ptr(xq), _ptr(xscale), M, K, _ptr(wq), _ptr(wscale), N,
+                                    _ptr(bias), _ptr(out), _stream()), "mxfp8_gemm_prequant")
+    return out
+
+
+def gelu_tanh(x: torch.Tensor, out=None):
+    _cuda(x, "x", torch.bfloat16)
+    if out is None:
+        out = torch.empty_like(x)
+    _check(_lib.mxfp8_gelu_tanh_bf16(_ptr(x), _ptr(out), x.numel(), _stream()), "mxfp8_gelu_tanh_bf16")
+    return out
+
+
+def device_status() -> int:
+    """Synchronize the current stream; 0 or the status a kernel recorded."""
+    return int(_lib.mxfp8_device_status(_stream()))

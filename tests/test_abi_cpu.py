@@ -1,0 +1,128 @@
+"""The C-ABI library loads and exports every symbol include/mxfp8.h declares;
+host-side argument checks reject bad calls before anything is launched.
+No GPU needed: none of these calls reaches the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mxfp8.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mxfp8_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from mxfp8_w8a8_quantized_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("mxfp8_quantize", "mxfp8_linear", "mxfp8_quantize_weight_f32", "mxfp8_gemm_prequant",
+                 "mxfp8_scale_bytes", "mxfp8_linear_workspace_bytes", "mxfp8_status_str",
+                 "mxfp8_gelu_tanh_bf16", "mxfp8_device_status"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/mxfp8.h but not exported"
+
+
+def test_binding_exports_match_header():
+    from mxfp8_w8a8_quantized_b200 import mxfp8
+    assert sorted(mxfp8.EXPORTS) == [n for n in declared_functions() if n in mxfp8.EXPORTS]
+    assert set(declared_functions()) <= set(mxfp8.EXPORTS) | set()
+
+
+def _sig(lib):
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    lib.mxfp8_scale_bytes.argtypes = [I64, I64, ctypes.c_int]
+    lib.mxfp8_scale_bytes.restype = ctypes.c_size_t
+    lib.mxfp8_linear_workspace_bytes.argtypes = [I64, I64]
+    lib.mxfp8_linear_workspace_bytes.restype = ctypes.c_size_t
+    lib.mxfp8_quantize.argtypes = [P, I64, I64, I64, P, P, ctypes.c_int, P]
+    lib.mxfp8_quantize_weight_f32.argtypes = [P, I64, I64, P, P, ctypes.c_int, P]
+    lib.mxfp8_linear.argtypes = [P, I64, I64, P, P, I64, P, P, P, ctypes.c_size_t, P]
+    lib.mxfp8_gemm_prequant.argtypes = [P, P, I64, I64, P, P, I64, P, P, P]
+    lib.mxfp8_gelu_tanh_bf16.argtypes = [P, P, I64, P]
+    lib.mxfp8_status_str.argtypes = [ctypes.c_int]
+    lib.mxfp8_status_str.restype = ctypes.c_char_p
+    return lib
+
+
+def test_sizes(lib):
+    L = _sig(lib)
+    assert L.mxfp8_scale_bytes(256, 512, 0) == 256 * 16
+    assert L.mxfp8_scale_bytes(256, 512, 1) == 2 * 4 * 512
+    assert L.mxfp8_scale_bytes(32760, 5120, 1) == 256 * 40 * 512   # ceil(32760/128) = 256
+    assert L.mxfp8_scale_bytes(1, 32, 1) == 512                    # padded to one atom
+    assert L.mxfp8_scale_bytes(10, 33, 1) == 0                     # K % 32 != 0
+    assert L.mxfp8_scale_bytes(-1, 32, 0) == 0
+    assert L.mxfp8_scale_bytes(10, 32, 7) == 0
+    ws = L.mxfp8_linear_workspace_bytes(32760, 5120)
+    assert ws == 32760 * 5120 + 256 * 40 * 512
+
+
+def test_status_strings(lib):
+    L = _sig(lib)
+    for s in range(6):
+        assert L.mxfp8_status_str(s).startswith(b"MXFP8_")
+    assert b"UNKNOWN" in L.mxfp8_status_str(99)
+
+
+FAKE = 0x10000  # a 16-byte aligned, never dereferenced address
+
+
+def test_argument_checks_return_before_launch(lib):
+    L = _sig(lib)
+    ARG, ALIGN, SHAPE = 1, 2, 3
+    # quantize
+    assert L.mxfp8_quantize(None, 4, 64, 64, FAKE, FAKE, 1, None) == ARG
+    assert L.mxfp8_quantize(FAKE, 4, 48, 48, FAKE, FAKE, 1, None) == SHAPE      # K % 32
+    assert L.mxfp8_quantize(FAKE, 4, 64, 32, FAKE, FAKE, 1, None) == ARG        # ldx < K
+    assert L.mxfp8_quantize(FAKE + 2, 4, 64, 64, FAKE, FAKE, 1, None) == ALIGN  # X misaligned
+    assert L.mxfp8_quantize(FAKE, 4, 64, 68, FAKE, FAKE, 1, None) == ALIGN      # row stride
+    assert L.mxfp8_quantize(FAKE, 4, 64, 64, FAKE, FAKE, 5, None) == ARG        # layout
+    assert L.mxfp8_quantize(FAKE, -1, 64, 64, FAKE, FAKE, 1, None) == ARG
+    assert L.mxfp8_quantize(FAKE, 0, 64, 64, FAKE, FAKE, 1, None) == 0          # empty: no-op
+    # weights
+    assert L.mxfp8_quantize_weight_f32(FAKE, 4, 40, FAKE, FAKE, 1, None) == SHAPE
+    # gemm
+    assert L.mxfp8_gemm_prequant(FAKE, FAKE, 4, 96, FAKE, FAKE, 16, None, FAKE, None) == SHAPE   # K % 128
+    assert L.mxfp8_gemm_prequant(FAKE, FAKE, 4, 128, FAKE, FAKE, 12, None, FAKE, None) == SHAPE  # N % 8
+    assert L.mxfp8_gemm_prequant(FAKE, FAKE, 4, 128, FAKE, FAKE, 16, FAKE + 8, FAKE, None) == ALIGN
+    assert L.mxfp8_gemm_prequant(FAKE, None, 4, 128, FAKE, FAKE, 16, None, FAKE, None) == ARG
+    assert L.mxfp8_gemm_prequant(FAKE, FAKE, 0, 128, FAKE, FAKE, 16, None, FAKE, None) == 0
+    assert L.mxfp8_gemm_prequant(FAKE, FAKE, 4, 128, FAKE, FAKE, 0, None, FAKE, None) == ARG
+    # linear: workspace too small, misaligned workspace
+    need = L.mxfp8_linear_workspace_bytes(4, 128)
+    assert L.mxfp8_linear(FAKE, 4, 128, FAKE, FAKE, 16, None, FAKE, FAKE, need - 1, None) == ARG
+    assert L.mxfp8_linear(FAKE, 4, 128, FAKE, FAKE, 16, None, FAKE, FAKE + 16, need, None) == ALIGN
+    assert L.mxfp8_linear(FAKE, 4, 100, FAKE, FAKE, 16, None, FAKE, FAKE, 1 << 20, None) == SHAPE
+    # gelu
+    assert L.mxfp8_gelu_tanh_bf16(FAKE, FAKE, 12, None) == SHAPE
+    assert L.mxfp8_gelu_tanh_bf16(FAKE, FAKE + 4, 16, None) == ALIGN
+    assert L.mxfp8_gelu_tanh_bf16(FAKE, FAKE, 0, None) == 0
+
+
+def test_product_fails_loudly_without_library(tmp_path, monkeypatch):
+    import importlib.util
+    import sys
+    src = os.path.join(ROOT, "mxfp8_w8a8_quantized_b200", "mxfp8.py")
+    # load a copy of the binding next to no library: the import must raise
+    dst = tmp_path / "mxfp8.py"
+    dst.write_text(open(src).read())
+    spec = importlib.util.spec_from_file_location("mxfp8_copy", str(dst))
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError):
+        spec.loader.exec_module(mod)
+    assert "mxfp8_copy" not in sys.modules
