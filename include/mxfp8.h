@@ -147,6 +147,40 @@ mxfp8_status mxfp8_gemm_prequant(const void *Xq, const void *Xscale, int64_t M, 
 mxfp8_status mxfp8_gelu_tanh_bf16(const void *X, void *Y, int64_t n, mxfp8_stream_t stream);
 
 /*
+ * mxfp8_linear for callers that cannot allocate device memory.  The pages
+ * have no counterpart of this entry point; it exists for users of this
+ * library.  mxfp8_linear needs a workspace for the quantized activations;
+ * some callers cannot provide one -- code running inside another runtime's
+ * launch hook where allocation is not allowed, or a process whose memory
+ * allocator already holds all of the GPU's memory, so that cudaMalloc (which
+ * also synchronizes the device) would fail or stall other streams.  This
+ * variant uses a fixed scratch array inside the library instead and
+ * allocates nothing (no cudaMalloc, no cudaFree, no allocating library call).
+ *
+ *   Same arguments, requirements and results as mxfp8_linear, minus the
+ *   workspace.  The activation codes must fit MXFP8_NOALLOC_MAX_CODE_BYTES
+ *   (M * K <= 32 MiB, e.g. M <= 6553 rows at K = 5120) and their scales
+ *   MXFP8_NOALLOC_MAX_SCALE_BYTES; larger problems return MXFP8_ERR_SHAPE
+ *   before anything is launched.
+ *   Memory: the scratch is a 34 MiB device array that every GPU which loads
+ *   the library keeps until the process exits.
+ *   First call on a device: looks up the scratch's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call before any stream capture.
+ *   Concurrency: all calls on a device share the one scratch array, which
+ *   keeps the last call's contents.  Calls whose work overlaps on the GPU
+ *   (different streams, or different host threads without ordering) race on
+ *   it and give wrong results; order them on one stream.  Nothing in the
+ *   scratch needs clearing between calls.
+ */
+#define MXFP8_NOALLOC_MAX_CODE_BYTES (32ll << 20)
+#define MXFP8_NOALLOC_MAX_SCALE_BYTES (2ll << 20)
+#define MXFP8_NOALLOC_SCRATCH_BYTES (MXFP8_NOALLOC_MAX_CODE_BYTES + MXFP8_NOALLOC_MAX_SCALE_BYTES)
+mxfp8_status mxfp8_linear_noalloc(const void *X, int64_t M, int64_t K,
+                                  const void *Wq, const void *Wscale, int64_t N,
+                                  const void *bias, void *Y, mxfp8_stream_t stream);
+
+/*
  * Synchronizes `stream`, then reads and clears the library's device status
  * word on the current device.  Returns MXFP8_ERR_TIMEOUT if a kernel gave up
  * a pipeline wait since the last call, MXFP8_ERR_CUDA if the stream reports

@@ -40,6 +40,8 @@ _lib.mxfp8_gemm_prequant.argtypes = [_P, _P, _I64, _I64, _P, _P, _I64, _P, _P, _
 _lib.mxfp8_gemm_prequant.restype = ctypes.c_int
 _lib.mxfp8_gelu_tanh_bf16.argtypes = [_P, _P, _I64, _P]
 _lib.mxfp8_gelu_tanh_bf16.restype = ctypes.c_int
+_lib.mxfp8_linear_noalloc.argtypes = [_P, _I64, _I64, _P, _P, _I64, _P, _P, _P]
+_lib.mxfp8_linear_noalloc.restype = ctypes.c_int
 _lib.mxfp8_device_status.argtypes = [_P]
 _lib.mxfp8_device_status.restype = ctypes.c_int
 
@@ -48,7 +50,7 @@ SF_TCGEN05 = 1
 
 EXPORTS = ("mxfp8_status_str", "mxfp8_scale_bytes", "mxfp8_quantize", "mxfp8_quantize_weight_f32",
            "mxfp8_linear_workspace_bytes", "mxfp8_linear", "mxfp8_gemm_prequant",
-           "mxfp8_gelu_tanh_bf16", "mxfp8_device_status")
+           "mxfp8_gelu_tanh_bf16", "mxfp8_device_status", "mxfp8_linear_noalloc")
 
 
 class MXFP8Error(RuntimeError):
@@ -127,6 +129,20 @@ def linear(x: torch.Tensor, wq: torch.Tensor, wscale: torch.Tensor, bias=None, o
         workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=x.device)
     _check(_lib.mxfp8_linear(_ptr(x), M, K, _ptr(wq), _ptr(wscale), N, _ptr(bias), _ptr(out),
                              _ptr(workspace), workspace.numel(), _stream()), "mxfp8_linear")
+    return out
+
+
+def linear_noalloc(x: torch.Tensor, wq: torch.Tensor, wscale: torch.Tensor, bias=None, out=None):
+    """As `linear`, for callers that cannot allocate device memory: the
+    library's fixed internal scratch replaces the workspace (M * K must fit
+    32 MiB).  Only `out` is allocated here, and only when it is not given."""
+    _cuda(x, "x", torch.bfloat16)
+    M, K = x.shape
+    N = wq.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _check(_lib.mxfp8_linear_noalloc(_ptr(x), M, K, _ptr(wq), _ptr(wscale), N, _ptr(bias), _ptr(out),
+                                     _stream()), "mxfp8_linear_noalloc")
     return out
 
 
