@@ -14,14 +14,15 @@
  * x * 2^-e (exact: a power-of-two multiply of a BF16/FP32 value).
  *
  * HBM-bound: 2 (BF16) or 4 (FP32) bytes read + 1 code byte + 1/32 scale byte
- * written per element.  Each warp handles row segments of 256 elements: every
- * lane loads 8 consecutive elements with 128-bit loads (fully coalesced 512 B
- * per warp load), 4 lanes form one 32-block and reduce amax with two
- * shuffle-xor steps, each lane packs 8 codes into one 8-byte store (coalesced
- * 256 B per warp), and scales are gathered into 32-bit words written straight
- * into the tensor-core scale layout (see include/mxfp8.h).  Four segments are
- * loaded before any is processed to keep several 16-byte loads in flight per
- * thread.
+ * written per element.  Each warp handles row segments of 512 elements: every
+ * lane loads 16 consecutive elements with two 128-bit loads (fully coalesced),
+ * two lanes form one 32-block and combine their amax with one shuffle, each
+ * lane writes its 16 codes with one 16-byte store (coalesced 512 B per warp),
+ * and scales are gathered into 32-bit words written straight into the
+ * tensor-core scale layout (see include/mxfp8.h).  Two segments are loaded
+ * before either is processed, keeping four 16-byte loads in flight per
+ * thread.  The row/segment walk has no division in the loop: the kernel is
+ * close to instruction-bound, so every per-element instruction counts.
  */
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
@@ -30,8 +31,14 @@
 
 namespace mx {
 
+#ifndef MX_QUNROLL
+#define MX_QUNROLL 2
+#endif
+#ifndef MX_QMINBLOCKS
+#define MX_QMINBLOCKS 1
+#endif
 constexpr int QTHREADS = 256;
-constexpr int QUNROLL = 4;
+constexpr int QUNROLL = MX_QUNROLL;     /* row segments in flight per warp */
 
 /* Scale byte from the bit pattern of amax as a binary32 (sign cleared). */
 __device__ __forceinline__ uint32_t scale_byte_from_amax(uint32_t abits)
@@ -55,120 +62,156 @@ __device__ __forceinline__ uint32_t pack4_e4m3(float a, float b, float c, float 
     return (uint32_t)lo | ((uint32_t)hi << 16);
 }
 
+/* 16 consecutive elements of one row: one lane's share of a row segment. */
 template <bool F32_IN>
-struct Seg8 {
-    uint4 v[F32_IN ? 2 : 1];
+struct Seg16 {
+    uint4 v[F32_IN ? 4 : 2];
 };
 
 template <bool F32_IN>
-__device__ __forceinline__ void load_seg8(Seg8<F32_IN> &s, const void *base, int64_t elem_off)
+__device__ __forceinline__ void load_seg16(Seg16<F32_IN> &s, const void *base, int64_t elem_off)
 {
     if constexpr (F32_IN) {
         const uint4 *p = reinterpret_cast<const uint4 *>(reinterpret_cast<const float *>(base) + elem_off);
-        s.v[0] = __ldcs(p);
-        s.v[1] = __ldcs(p + 1);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            s.v[i] = __ldcs(p + i);
     } else {
         const uint4 *p = reinterpret_cast<const uint4 *>(reinterpret_cast<const uint16_t *>(base) + elem_off);
         s.v[0] = __ldcs(p);
+        s.v[1] = __ldcs(p + 1);
     }
 }
 
-/* The 8 elements as floats, and the max of their magnitudes as binary32 bits. */
+/* max |x| of the 16 elements, as the bit pattern of a binary32 (sign cleared) */
 template <bool F32_IN>
-__device__ __forceinline__ uint32_t unpack_seg8(const Seg8<F32_IN> &s, float (&f)[8])
+__device__ __forceinline__ uint32_t amax_seg16(const Seg16<F32_IN> &s)
 {
-    uint32_t amax = 0;
     if constexpr (F32_IN) {
-        const uint32_t w[8] = {s.v[0].x, s.v[0].y, s.v[0].z, s.v[0].w, s.v[1].x, s.v[1].y, s.v[1].z, s.v[1].w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            f[i] = __uint_as_float(w[i]);
-            amax = max(amax, w[i] & 0x7FFFFFFFu);
-        }
-    } else {
-        const uint32_t w[4] = {s.v[0].x, s.v[0].y, s.v[0].z, s.v[0].w};
+        uint32_t m = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            uint32_t lo = w[i] << 16, hi = w[i] & 0xFFFF0000u;
-            f[2 * i] = __uint_as_float(lo);
-            f[2 * i + 1] = __uint_as_float(hi);
-            amax = max(amax, max(lo & 0x7FFFFFFFu, hi & 0x7FFFFFFFu));
+            m = max(m, s.v[i].x & 0x7FFFFFFFu);
+            m = max(m, s.v[i].y & 0x7FFFFFFFu);
+            m = max(m, s.v[i].z & 0x7FFFFFFFu);
+            m = max(m, s.v[i].w & 0x7FFFFFFFu);
         }
+        return m;
+    } else {
+        /* non-negative BF16 bit patterns order like the values (NaN above
+         * Inf above every finite value): packed unsigned 16-bit max */
+        const uint32_t k = 0x7FFF7FFFu;
+        uint32_t a = __vmaxu2(s.v[0].x & k, s.v[0].y & k);
+        uint32_t b = __vmaxu2(s.v[0].z & k, s.v[0].w & k);
+        uint32_t c = __vmaxu2(s.v[1].x & k, s.v[1].y & k);
+        uint32_t d = __vmaxu2(s.v[1].z & k, s.v[1].w & k);
+        uint32_t m = __vmaxu2(__vmaxu2(a, b), __vmaxu2(c, d));
+        return max(m << 16, m & 0xFFFF0000u);
     }
-    return amax;
+}
+
+/* 16 elements times 2^-e (exact) -> 16 E4M3 codes */
+template <bool F32_IN>
+__device__ __forceinline__ uint4 codes_seg16(const Seg16<F32_IN> &s, float m)
+{
+    uint32_t out[4];
+    if constexpr (F32_IN) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            out[i] = pack4_e4m3(__uint_as_float(s.v[i].x) * m, __uint_as_float(s.v[i].y) * m,
+                                __uint_as_float(s.v[i].z) * m, __uint_as_float(s.v[i].w) * m);
+    } else {
+        const uint32_t w[8] = {s.v[0].x, s.v[0].y, s.v[0].z, s.v[0].w, s.v[1].x, s.v[1].y, s.v[1].z, s.v[1].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            out[i] = pack4_e4m3(__uint_as_float(w[2 * i] << 16) * m, __uint_as_float(w[2 * i] & 0xFFFF0000u) * m,
+                                __uint_as_float(w[2 * i + 1] << 16) * m,
+                                __uint_as_float(w[2 * i + 1] & 0xFFFF0000u) * m);
+    }
+    return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
 /*
  * X [M, K] (row stride ldx elements) -> Q [M, K] codes, S scales.
- * Work unit = (row r, segment j of 256 elements); rows r in [M, Mrows) only
- * write zero scale padding (tensor-core layout).
+ * Work unit = (row r, segment j of 512 elements); lane l covers elements
+ * 16l .. 16l+15 of the segment, so lanes 2b and 2b+1 hold block b.  Rows r in
+ * [M, Mrows) only write zero scale padding (tensor-core layout).
  */
 template <bool F32_IN, bool SF_TC>
-__global__ void __launch_bounds__(QTHREADS) mx_quantize_kernel(const void *__restrict__ X, int64_t M, int64_t K,
-                                                               int64_t ldx, uint8_t *__restrict__ Q,
-                                                               uint8_t *__restrict__ S, int64_t Mrows,
-                                                               int64_t nseg, int64_t kgroups)
+__global__ void __launch_bounds__(QTHREADS, MX_QMINBLOCKS) mx_quantize_kernel(const void *__restrict__ X, int64_t M,
+                                                                              int64_t K, int64_t ldx,
+                                                                              uint8_t *__restrict__ Q,
+                                                                              uint8_t *__restrict__ S, int64_t Mrows,
+                                                                              int64_t nseg, int64_t kgroups)
 {
     const int lane = threadIdx.x & 31;
     const int64_t warp0 = ((int64_t)blockIdx.x * QTHREADS + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * QTHREADS) >> 5;
     const int64_t units = Mrows * nseg;
-    const int64_t nblocks = K >> 5;
+    const int nblocks = (int)(K >> 5);
+    /* Walk the (row, segment) space without dividing in the loop: one
+     * division up front, then carry-propagating increments. */
+    const int64_t stride = nwarps * QUNROLL;
+    const int nseg32 = (int)nseg;
+    const int stride_r = (int)(stride / nseg), stride_j = (int)(stride - (int64_t)stride_r * nseg);
+    int64_t u0 = warp0 * QUNROLL;
+    int r0 = (int)(u0 / nseg), j0 = (int)(u0 - (int64_t)r0 * nseg);
+    const int M32 = (int)M, K32 = (int)K;
 
-    for (int64_t u0 = warp0 * QUNROLL; u0 < units; u0 += nwarps * QUNROLL) {
-        Seg8<F32_IN> seg[QUNROLL];
-        int64_t row[QUNROLL], k0[QUNROLL];
+    for (; u0 < units; u0 += stride) {
+        Seg16<F32_IN> seg[QUNROLL];
+        int row[QUNROLL], k0[QUNROLL];
         bool valid[QUNROLL];
+        {
+            int r = r0, j = j0;
 #pragma unroll
-        for (int i = 0; i < QUNROLL; ++i) {
-            const int64_t u = u0 + i;
-            row[i] = u / nseg;
-            k0[i] = (u - row[i] * nseg) * 256 + lane * 8;
-            valid[i] = (u < units) && (row[i] < M) && (k0[i] < K);
-            if (valid[i])
-                load_seg8<F32_IN>(seg[i], X, row[i] * ldx + k0[i]);
+            for (int i = 0; i < QUNROLL; ++i) {
+                row[i] = r;
+                k0[i] = j * 512 + lane * 16;
+                valid[i] = (u0 + i < units) && (r < M32) && (k0[i] < K32);
+                if (valid[i])
+                    load_seg16<F32_IN>(seg[i], X, (int64_t)r * ldx + k0[i]);
+                if (++j == nseg32) {
+                    j = 0;
+                    ++r;
+                }
+            }
+        }
+        r0 += stride_r;
+        j0 += stride_j;
+        if (j0 >= nseg32) {
+            j0 -= nseg32;
+            ++r0;
         }
 #pragma unroll
         for (int i = 0; i < QUNROLL; ++i) {
             if (u0 + i >= units) /* warp-uniform */
                 break;
-            float f[8];
-            uint32_t amax = 0;
-            if (valid[i])
-                amax = unpack_seg8<F32_IN>(seg[i], f);
+            uint32_t amax = valid[i] ? amax_seg16<F32_IN>(seg[i]) : 0u;
             amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-            amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
             const uint32_t sb = valid[i] ? scale_byte_from_amax(amax) : 0u;
             if (valid[i]) {
-                uint2 out;
-                if (sb == 0xFFu) {
-                    out = make_uint2(0x7F7F7F7Fu, 0x7F7F7F7Fu);
-                } else {
-                    const float m = inv_scale(sb);
-                    out.x = pack4_e4m3(f[0] * m, f[1] * m, f[2] * m, f[3] * m);
-                    out.y = pack4_e4m3(f[4] * m, f[5] * m, f[6] * m, f[7] * m);
-                }
-                *reinterpret_cast<uint2 *>(Q + row[i] * K + k0[i]) = out;
+                const uint4 out = (sb == 0xFFu) ? make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu)
+                                                : codes_seg16<F32_IN>(seg[i], inv_scale(sb));
+                *reinterpret_cast<uint4 *>(Q + (int64_t)row[i] * K + k0[i]) = out;
             }
             if constexpr (SF_TC) {
-                /* lanes 0,4,8,12 hold blocks 8j..8j+3, lanes 16..28 blocks 8j+4..8j+7 */
-                const int base = lane & 16;
-                const uint32_t w = __shfl_sync(0xFFFFFFFFu, sb, base) |
-                                   (__shfl_sync(0xFFFFFFFFu, sb, base + 4) << 8) |
-                                   (__shfl_sync(0xFFFFFFFFu, sb, base + 8) << 16) |
-                                   (__shfl_sync(0xFFFFFFFFu, sb, base + 12) << 24);
-                if ((lane & 15) == 0) {
-                    const int64_t r = row[i];
-                    const int64_t kb = ((k0[i] - lane * 8) >> 5) + (lane >> 2); /* first block of this word */
+                /* word g (lanes 8g .. 8g+7) = blocks 16j + 4g .. 16j + 4g + 3 */
+                const uint32_t w = sb | (__shfl_down_sync(0xFFFFFFFFu, sb, 2) << 8) |
+                                   (__shfl_down_sync(0xFFFFFFFFu, sb, 4) << 16) |
+                                   (__shfl_down_sync(0xFFFFFFFFu, sb, 6) << 24);
+                if ((lane & 7) == 0) {
+                    const int r = row[i];
+                    const int kb = ((k0[i] - lane * 16) >> 5) + (lane >> 1); /* first block of this word */
                     if (kb < nblocks) {
-                        const int64_t off = (((r >> 7) * kgroups + (kb >> 2)) << 9) + ((r & 31) << 4) +
+                        const int64_t off = ((((int64_t)(r >> 7)) * kgroups + (kb >> 2)) << 9) + ((r & 31) << 4) +
                                             (((r >> 5) & 3) << 2);
                         *reinterpret_cast<uint32_t *>(S + off) = w;
                     }
                 }
             } else {
-                if (valid[i] && (lane & 3) == 0)
-                    S[row[i] * nblocks + (k0[i] >> 5)] = (uint8_t)sb;
+                if (valid[i] && (lane & 1) == 0)
+                    S[(int64_t)row[i] * nblocks + (k0[i] >> 5)] = (uint8_t)sb;
             }
         }
     }
@@ -223,7 +266,7 @@ cudaError_t launch_quantize(const void *X, bool f32_in, int64_t M, int64_t K, in
                             bool sf_tc, cudaStream_t stream)
 {
     const int64_t Mrows = sf_tc ? ((M + 127) / 128) * 128 : M;
-    const int64_t nseg = (K + 255) / 256;
+    const int64_t nseg = (K + 511) / 512;
     const int64_t kgroups = (K / 32 + 3) / 4;
     const int64_t units = Mrows * nseg;
     if (units == 0)
