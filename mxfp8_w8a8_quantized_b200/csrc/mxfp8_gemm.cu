@@ -22,7 +22,7 @@
  *   issues the MMAs for the pair.
  *  SINGLE: one CTA per SM, 128 x 256 tiles, tcgen05.mma.cta_group::1.
  *
- * Roles (320 threads per CTA):
+ * Roles (352 threads per CTA):
  *   warp 0       TMA producer: per 128-wide K step, A and B tiles (tiled TMA,
  *                128-byte swizzle) and their scale atoms (512 B per 128
  *                rows, 3-D tiled TMA) into a multi-stage smem ring guarded
@@ -34,13 +34,22 @@
  *                K step picked by the instruction descriptor's scale-factor
  *                ID; tcgen05.commit frees the stage (in both CTAs) and, after
  *                the tile, signals the epilogues.
+ *   warp 10      (leader CTA of a pair) copies each stage's scales to TMEM
+ *                with the pair-wide tcgen05.cp and signals the MMA thread
+ *                through an mbarrier: that copy stalls the thread issuing it,
+ *                which must not be the one that keeps the tensor core fed.
  *   warps 2..9   epilogue: each warp owns one 32-lane TMEM sub-partition and
  *                half the columns; it drains its 32 x 128 FP32 block in one
  *                tcgen05.ld, releases the accumulator to the MMA thread at
- *                once, then adds the bias, rounds to BF16 and stores (rows
- *                >= M and columns >= N masked) while the next tile's MMAs run.
- * Scale columns in TMEM are per stage, so a scale copy never overwrites
- * scales an earlier, still running MMA reads.  Every wait is bounded: on
+ *                once, then adds the bias, rounds to BF16 and writes 32 x 32
+ *                boxes through a swizzled smem buffer with TMA stores
+ *                (clipped at M and N) while the next tile's MMAs run.
+ * The shared-memory data path is the scarce resource: TMA writes each stage
+ * and the tensor core reads it (~130 B/clock per SM at full MMA rate), so
+ * everything else is kept off it -- waits sleep in mbarrier.try_wait instead
+ * of spinning, and the output leaves through bulk TMA stores rather than
+ * per-row global stores.  Scale columns in TMEM are per stage, so a scale
+ * copy never overwrites scales an earlier, still running MMA reads.  Every wait is bounded: on
  * timeout the kernel records MXFP8_ERR_TIMEOUT in a device status word,
  * drains its own MMAs, frees TMEM and returns.
  */
@@ -57,10 +66,25 @@ namespace mx {
 
 constexpr int BK = 128; /* bytes = E4M3 elements per K step */
 constexpr int EPI_WARPS = 8;
-constexpr int GEMM_THREADS = (2 + EPI_WARPS) * 32;
+constexpr int SF_WARP = 2 + EPI_WARPS; /* copies scales to TMEM (CTA-pair variant) */
+constexpr int GEMM_THREADS = (3 + EPI_WARPS) * 32;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0; /* 256 FP32 columns */
 constexpr int RASTER_GROUP = 8; /* M tiles walked together for L2 reuse */
+#ifndef MX_PREFETCH_KB
+#define MX_PREFETCH_KB 0
+#endif
+#ifndef MX_SUSPEND_PIPE
+#define MX_SUSPEND_PIPE 1000000
+#endif
+#ifndef MX_SUSPEND_EPI
+#define MX_SUSPEND_EPI 1000000
+#endif
+/* mbarrier.try_wait suspend-time hints (ns): the producer and MMA threads wait
+ * briefly and often, the epilogue warps for a whole tile */
+constexpr uint32_t SUSPEND_PIPE = MX_SUSPEND_PIPE;
+constexpr uint32_t SUSPEND_EPI = MX_SUSPEND_EPI;
+constexpr int PREFETCH_KB = MX_PREFETCH_KB; /* K steps the L2 prefetch runs ahead of the loads (0 = off) */
 constexpr uint32_t ST_TIMEOUT = 1u;
 
 template <bool PAIR>
@@ -82,14 +106,17 @@ struct Cfg {
     static constexpr uint32_t OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr uint32_t OFF_SFA = OFF_B + STAGES * B_BYTES;
     static constexpr uint32_t OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
-    static constexpr uint32_t OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
-    static constexpr uint32_t NUM_BARS = 2 * STAGES + 3; /* full[], empty[], tmem_full, tmem_empty, drain */
+    static constexpr uint32_t OFF_EPI = OFF_SFB + STAGES * SFB_BYTES; /* 1 KiB aligned */
+    static constexpr uint32_t EPI_BUF = 32 * 32 * 2;                    /* 32 rows x 32 BF16 */
+    static constexpr uint32_t OFF_BAR = OFF_EPI + EPI_WARPS * EPI_BUF;
+    static constexpr uint32_t NUM_BARS = 3 * STAGES + 3; /* full[], empty[], sf_full[], tmem_full, tmem_empty, drain */
     static constexpr uint32_t OFF_TMEMPTR = OFF_BAR + NUM_BARS * 8;
     static constexpr uint32_t OFF_ABORT = OFF_TMEMPTR + 4;
     static constexpr uint32_t SMEM_USED = OFF_TMEMPTR + 16;
     static constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024; /* slack to align the base to 1 KiB */
     static constexpr uint32_t TEMPTY_ARRIVALS = EPI_WARPS * (PAIR ? 2u : 1u);
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+    static_assert(OFF_EPI % 1024 == 0, "staging buffers must be swizzle-atom aligned");
 };
 
 __device__ unsigned int g_mx_status = 0;
@@ -119,16 +146,14 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int &mb
  * CTA's abort flag, so the other roles stop waiting too.
  */
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, unsigned long long limit_ns,
-                                             volatile uint32_t *abort_flag)
+                                             volatile uint32_t *abort_flag, uint32_t suspend_ns = SUSPEND_PIPE)
 {
-    if (mbar_try_wait(bar, parity))
+    if (mbar_try_wait(bar, parity, suspend_ns))
         return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-#pragma unroll 1
-        for (int i = 0; i < 256; ++i)
-            if (mbar_try_wait(bar, parity))
-                return true;
+        if (mbar_try_wait(bar, parity, suspend_ns))
+            return true;
         if (*abort_flag)
             return false;
         if (globaltimer_ns() - t0 > limit_ns) {
@@ -143,7 +168,7 @@ template <bool PAIR>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
-                      const GemmParams p)
+                      const __grid_constant__ CUtensorMap tmap_y, const GemmParams p)
 {
     using C = Cfg<PAIR>;
     extern __shared__ uint8_t smem_raw[];
@@ -159,7 +184,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
     const uint32_t bar_full = sbase + C::OFF_BAR;          /* + 8 s */
     const uint32_t bar_empty = bar_full + C::STAGES * 8;   /* + 8 s */
-    const uint32_t bar_tfull = bar_empty + C::STAGES * 8;
+    const uint32_t bar_sffull = bar_empty + C::STAGES * 8; /* + 8 s */
+    const uint32_t bar_tfull = bar_sffull + C::STAGES * 8;
     const uint32_t bar_tempty = bar_tfull + 8;
     const uint32_t bar_drain = bar_tempty + 8;
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + C::OFF_TMEMPTR);
@@ -170,6 +196,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(bar_full + 8 * s, 1);
             mbar_init(bar_empty + 8 * s, 1);
+            mbar_init(bar_sffull + 8 * s, 1);
         }
         mbar_init(bar_tfull, 1);
         mbar_init(bar_tempty, C::TEMPTY_ARRIVALS);
@@ -225,6 +252,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     const uint32_t dB = sbase + C::OFF_B + s * C::B_BYTES;
                     const uint32_t dSA = sbase + C::OFF_SFA + s * C::SFA_BYTES;
                     const uint32_t dSB = sbase + C::OFF_SFB + s * C::SFB_BYTES;
+                    if (PREFETCH_KB > 0) {
+                        /* operand boxes PREFETCH_KB K steps ahead (in this tile
+                         * or the next one of this CTA) go to L2 now, so that
+                         * the stage loads hit L2 instead of waiting on DRAM */
+                        int pkb = kb + PREFETCH_KB, pt = t;
+                        if (pkb >= KB) {
+                            pkb -= KB;
+                            pt += tstep;
+                        }
+                        if (pt < num_tiles && pkb < KB) {
+                            int pmb = mb, pnb = nb;
+                            if (pt != t)
+                                tile_coords(pt, p.num_m, p.num_n, pmb, pnb);
+                            const int pra = pmb * C::TILE_M + (int)(rank * 128u);
+                            const int prb = pnb * C::TILE_N + (int)(rank * C::B_ROWS);
+                            if (pra < p.M)
+                                tma_prefetch_2d(&tmap_a, pkb * BK, pra);
+                            if (prb < p.N)
+                                tma_prefetch_2d(&tmap_b, pkb * BK, prb);
+                        }
+                    }
                     if constexpr (PAIR) {
                         const uint32_t lead = mapa_shared(full, 0u);
                         tma_load_2d_pair(dA, &tmap_a, kb * BK, rowA, lead);
@@ -254,7 +302,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 tc_fence_after();
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const uint32_t s = it % C::STAGES, ph = (it / C::STAGES) & 1u;
-                    if (!wait_bounded(bar_full + 8 * s, ph, lim, abort_flag)) {
+                    if (!wait_bounded(bar_full + 8 * s, ph, lim, abort_flag) ||
+                        (PAIR && !wait_bounded(bar_sffull + 8 * s, ph, lim, abort_flag))) {
                         ok = false;
                         break;
                     }
@@ -266,9 +315,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     const uint64_t adesc = desc_kmajor_sw128(sbase + C::OFF_A + s * C::A_BYTES);
                     const uint64_t bdesc = desc_kmajor_sw128(sbase + C::OFF_B + s * C::B_BYTES);
                     if constexpr (PAIR) {
-                        tc_cp_32x128b_warpx4_pair(tsfa, desc_sf_32x16(sfa_s));
-                        tc_cp_32x128b_warpx4_pair(tsfb, desc_sf_32x16(sfb_s));
-                        tc_cp_32x128b_warpx4_pair(tsfb + 4, desc_sf_32x16(sfb_s + 512u));
+                        /* scales were copied to TMEM by the scale warp */
+                        (void)sfa_s;
+                        (void)sfb_s;
 #pragma unroll
                         for (int k = 0; k < BK / 32; ++k)
                             tc_mma_mxf8_pair(tmem + ACC_COL, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k),
@@ -308,6 +357,35 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 (void)wait_bounded(bar_drain, 0u, lim, &own);
             }
         }
+    } else if (warp == SF_WARP) {
+        /* ------------------------------------------------ scale copies */
+        /* The pair-wide tcgen05.cp holds up the thread that issues it, so it
+         * is issued here, one stage at a time, and the MMA thread only waits
+         * for its completion (sf_full), never for the copy itself. */
+        if (PAIR && lane == 0 && rank == 0) {
+            uint32_t it = 0;
+            for (int t = tile0; t < num_tiles; t += tstep) {
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const uint32_t s = it % C::STAGES, ph = (it / C::STAGES) & 1u;
+                    if (!wait_bounded(bar_full + 8 * s, ph, lim, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t tsfa = tmem + C::SFA_COL + 4 * s;
+                    const uint32_t tsfb = tmem + C::SFB_COL + 8 * s;
+                    const uint32_t sfa_s = sbase + C::OFF_SFA + s * C::SFA_BYTES;
+                    const uint32_t sfb_s = sbase + C::OFF_SFB + s * C::SFB_BYTES;
+                    tc_cp_32x128b_warpx4_pair(tsfa, desc_sf_32x16(sfa_s));
+                    tc_cp_32x128b_warpx4_pair(tsfb, desc_sf_32x16(sfb_s));
+                    tc_cp_32x128b_warpx4_pair(tsfb + 4, desc_sf_32x16(sfb_s + 512u));
+                    tc_commit_pair(bar_sffull + 8 * s, (uint16_t)0x1);
+                }
+                if (!ok)
+                    break;
+            }
+        }
     } else {
         /* ------------------------------------------------ epilogue */
         const int q = warp & 3;            /* TMEM sub-partition this warp may read */
@@ -319,7 +397,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             tile_coords(t, p.num_m, p.num_n, mb, nb);
             /* every lane polls; the vote keeps the warp converged for the
              * .sync.aligned TMEM load and makes the outcome warp-uniform */
-            const bool got = wait_bounded(bar_tfull, tl & 1u, lim, abort_flag);
+            const bool got = wait_bounded(bar_tfull, tl & 1u, lim, abort_flag, SUSPEND_EPI);
             if (!__all_sync(0xFFFFFFFFu, got))
                 break;
             tc_fence_after();
@@ -334,38 +412,57 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     mbar_arrive(bar_tempty);
             }
 
-            const int row = mb * C::TILE_M + (int)(rank * 128u) + 32 * q + lane;
+            /* bias + BF16 rounding, 32 columns at a time, staged through a
+             * 64-byte-swizzled smem box and written by one TMA store per
+             * warp: scattered per-row global stores would occupy the L1 /
+             * shared-memory data path that feeds the tensor core. */
+            const int row0 = mb * C::TILE_M + (int)(rank * 128u) + 32 * q;
             const int col0 = nb * C::TILE_N + h * 128;
-            if (row < p.M) {
-                __nv_bfloat16 *yrow = p.Y + (size_t)row * p.N;
+            const uint32_t buf = sbase + C::OFF_EPI + (uint32_t)(warp - 2) * C::EPI_BUF;
+            const uint32_t rowbase = buf + (uint32_t)lane * 64u;
+            const uint32_t swz = ((uint32_t)lane >> 1) & 3u;
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const int col = col0 + 8 * c;
-                    if (col < p.N) {
-                        float b[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                        if (p.bias) {
-                            const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(p.bias + col));
-                            const __half2 *bh = reinterpret_cast<const __half2 *>(&bv);
+            for (int c = 0; c < 4; ++c) {
+                const int colc = col0 + 32 * c;
+                if (row0 >= p.M || colc >= p.N) /* whole box outside Y: nothing to store */
+                    continue;
+                if (lane == 0)
+                    bulk_wait_group_read0(); /* previous box has left the buffer */
+                __syncwarp();
 #pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const float2 f2 = __half22float2(bh[j]);
-                                b[2 * j] = f2.x;
-                                b[2 * j + 1] = f2.y;
-                            }
-                        }
-                        uint32_t o[4];
+                for (int j8 = 0; j8 < 4; ++j8) {
+                    const int col = colc + 8 * j8;
+                    float b[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    if (p.bias && col < p.N) {
+                        const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(p.bias + col));
+                        const __half2 *bh = reinterpret_cast<const __half2 *>(&bv);
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
-                            __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(acc[8 * c + 2 * j]) + b[2 * j],
-                                                                     __uint_as_float(acc[8 * c + 2 * j + 1]) +
-                                                                         b[2 * j + 1]);
-                            o[j] = *reinterpret_cast<uint32_t *>(&v);
+                            const float2 f2 = __half22float2(bh[j]);
+                            b[2 * j] = f2.x;
+                            b[2 * j + 1] = f2.y;
                         }
-                        *reinterpret_cast<uint4 *>(yrow + col) = make_uint4(o[0], o[1], o[2], o[3]);
                     }
+                    uint32_t o[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int a = 32 * c + 8 * j8 + 2 * j;
+                        __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(acc[a]) + b[2 * j],
+                                                                 __uint_as_float(acc[a + 1]) + b[2 * j + 1]);
+                        o[j] = *reinterpret_cast<uint32_t *>(&v);
+                    }
+                    st_shared_v4(rowbase + ((((uint32_t)j8) ^ swz) << 4), o[0], o[1], o[2], o[3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmap_y, colc, row0, buf);
+                    bulk_commit_group();
                 }
             }
         }
+        if (lane == 0)
+            bulk_wait_group0(); /* stores complete before the CTA exits */
     }
 
     tc_fence_before();
@@ -434,6 +531,22 @@ static bool make_scale_map(CUtensorMap *m, const void *base, int64_t rows, int64
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+/* BF16 output Y [M, N]: box 32 columns x 32 rows, 64-byte swizzle (the
+ * epilogue's staging layout); stores are clipped at M and N. */
+static bool make_output_map(CUtensorMap *m, void *base, int64_t M, int64_t N)
+{
+    PFN_encodeTiled enc = get_encode_fn();
+    if (!enc)
+        return false;
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)(N * 2)};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct DevInfo {
     bool init = false;
     int sms = 148;
@@ -459,7 +572,8 @@ static DevInfo *dev_info()
 
 template <bool PAIR>
 static cudaError_t launch_variant(const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorMap &msa,
-                                  const CUtensorMap &msb, const GemmParams &p, int grid, cudaStream_t stream)
+                                  const CUtensorMap &msb, const CUtensorMap &my, const GemmParams &p, int grid,
+                                  cudaStream_t stream)
 {
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
@@ -475,7 +589,7 @@ static cudaError_t launch_variant(const CUtensorMap &ma, const CUtensorMap &mb, 
         cfg.attrs = attr;
         cfg.numAttrs = 1;
     }
-    return cudaLaunchKernelEx(&cfg, mxfp8_gemm_kernel<PAIR>, ma, mb, msa, msb, p);
+    return cudaLaunchKernelEx(&cfg, mxfp8_gemm_kernel<PAIR>, ma, mb, msa, msb, my, p);
 }
 
 /* Whether the CTA-pair variant is used: on unless MXFP8_GEMM_PAIR=0. */
@@ -541,9 +655,9 @@ int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void
     }
 
     const uint32_t b_rows = pair ? Cfg<true>::B_ROWS : Cfg<false>::B_ROWS;
-    CUtensorMap ma, mb, msa, msb;
+    CUtensorMap ma, mb, msa, msb, my;
     if (!make_operand_map(&ma, Xq, M, K, 128) || !make_operand_map(&mb, Wq, N, K, b_rows) ||
-        !make_scale_map(&msa, Xs, M, K, 1) || !make_scale_map(&msb, Ws, N, K, 2))
+        !make_scale_map(&msa, Xs, M, K, 1) || !make_scale_map(&msb, Ws, N, K, 2) || !make_output_map(&my, Y, M, N))
         return 1;
     GemmParams p;
     p.bias = static_cast<const __half *>(bias);
@@ -560,12 +674,12 @@ int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void
         int clusters = d->max_pair_clusters;
         if (clusters > tiles)
             clusters = tiles;
-        e = launch_variant<true>(ma, mb, msa, msb, p, 2 * clusters, stream);
+        e = launch_variant<true>(ma, mb, msa, msb, my, p, 2 * clusters, stream);
     } else {
         int grid = d->sms;
         if (grid > tiles)
             grid = tiles;
-        e = launch_variant<false>(ma, mb, msa, msb, p, grid, stream);
+        e = launch_variant<false>(ma, mb, msa, msb, my, p, grid, stream);
     }
     if (e != cudaSuccess) {
         *err = e;
