@@ -222,7 +222,11 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t a, uint32_t rank)
 /* arrive on an mbarrier that may live in another CTA of the cluster */
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
 {
+#ifdef MX_ARRIVE_RELEASE_CLUSTER
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+#else
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+#endif
 }
 __device__ __forceinline__ void cluster_sync_all()
 {
