@@ -2,26 +2,25 @@
 """Benchmark of the MXFP8 W8A8 linear layer on B200.
 
 One step = one pass of the whole hot path over one batch: dynamic MX
-quantization of the BF16 activations (one kernel) and the block-scaled
-tcgen05 GEMM with the F16-bias / BF16 epilogue (one kernel).  Weights are
-quantized once, offline, before timing.  Default workload: the Wan2.2 A14B
-self-attention Q projection at 480x832, 81 frames (M = 32760 tokens,
-K = N = 5120).
+quantization of every BF16 activation and the block-scaled tcgen05 GEMM
+with its F16-bias / BF16 epilogue for every linear of the workload (plus the
+GELU between the FFN linears).  Weights are quantized once, offline, before
+timing.  Default workload: the Wan2.2 A14B self-attention Q projection at
+480x832, 81 frames (M = 32760 tokens, K = N = 5120).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME]
 
-Prints ONE JSON line (rank 0).  `value` is whole-job TFLOP/s (2*M*N*K per
-step per GPU, all GPUs, divided by the slowest rank's device time).  Under
-torchrun each rank runs an independent replica (weak scaling, no data-path
-collective).  `--impl reference` times the CPU oracle on host cores on a
-bounded sample of the same workload.
+Prints ONE JSON line (rank 0).  `value` is whole-job TFLOP/s (2*M*N*K summed
+over the step's linears, over all GPUs, divided by the slowest rank's device
+time).  Under torchrun every rank runs an independent replica (weak scaling,
+no data-path collective).  `--impl reference` times the CPU oracle on host
+cores on a bounded sample of the same workload.
 """
 import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -37,37 +36,24 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FP8_OVER_BF16 = 2.0  # nominal dense ratio: 4.5 PF/s FP8 vs 2.25 PF/s BF16
 L2_FLUSH_BYTES = 256 << 20
+WORKLOADS = ["c1_q_proj_480p", "c0_small", "ffn0_832x1104", "ffn2_832x1104",
+             "c2_ffn_pair_832x1104", "c3_block_832x1104", "c4_step_832x1104"]
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="c1_q_proj_480p",
-                    choices=["c0_small", "c1_q_proj_480p", "ffn0_832x1104", "ffn2_832x1104"])
+    ap.add_argument("--workload", default=WORKLOADS[0], choices=WORKLOADS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
-    return ap.parse_args()
-
-
-def workload_shape(name):
-    from mxfp8_w8a8_quantized_b200 import synth
-    if name == "c0_small":
-        return dict(M=256, K=512, N=512, seed=0, desc="single linear 256x512x512")
-    if name == "c1_q_proj_480p":
-        return dict(M=synth.TOKENS_480P, K=synth.HIDDEN, N=synth.HIDDEN, seed=1,
-                    desc="Wan2.2 A14B attn1.to_q at 480x832, 81 frames (21x30x52 tokens)")
-    if name == "ffn0_832x1104":
-        return dict(M=synth.TOKENS_832x1104, K=synth.HIDDEN, N=synth.FFN, seed=2,
-                    desc="Wan2.2 A14B ffn.net.0.proj at 832x1104, 81 frames")
-    if name == "ffn2_832x1104":
-        return dict(M=synth.TOKENS_832x1104, K=synth.FFN, N=synth.HIDDEN, seed=2,
-                    desc="Wan2.2 A14B ffn.net.2 at 832x1104, 81 frames")
-    raise ValueError(name)
+    ap.add_argument("--reference-seconds", type=float, default=150.0,
+                    help="CPU time budget of the reference arm (warm-up + timed steps)")
+    return ap.parse_args(argv)
 
 
 def load_peaks():
@@ -79,36 +65,44 @@ def load_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
-# ---------------------------------------------------------------- distributed
-def dist_setup(n_gpus):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
-    return world, rank, local
+# ---------------------------------------------------------------- ranks
+class Ranks:
+    """World / rank bookkeeping; collectives only for the barrier and the
+    max over ranks (no data-path collective).  Works with NCCL (GPU tensors)
+    and gloo (CPU tensors)."""
 
+    def __init__(self, backend=None, device=None):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.device = device
+        self.dist = None
+        if self.world > 1 and backend is not None:
+            import datetime
 
-def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+            import torch.distributed as dist
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            kw = dict(timeout=datetime.timedelta(seconds=120))
+            if backend == "nccl":
+                kw["device_id"] = device
+            dist.init_process_group(backend, **kw)
+            self.dist = dist
 
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
 
-def max_over_ranks(world, v):
-    if world == 1:
-        return v
-    import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    def max(self, v: float) -> float:
+        if self.dist is None:
+            return v
+        dev = self.device if (self.device is not None and self.dist.get_backend() == "nccl") else "cpu"
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.dist is not None:
+            self.dist.destroy_process_group()
 
 
 # ---------------------------------------------------------------- clocks
@@ -164,76 +158,282 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(self.samples)}
 
 
+# ---------------------------------------------------------------- timing
+class KernelTimer:
+    """CUDA events around each library call of a step, on the launching
+    stream: per-kind device time (GEMM, quantizer, GELU)."""
+
+    def __init__(self, stream):
+        self.stream = stream
+        self.events = []          # (kind, start, end)
+        self.on = False
+
+    def __call__(self, kind, fn, *a, **kw):
+        if not self.on:
+            return fn(*a, **kw)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(self.stream)
+        r = fn(*a, **kw)
+        e.record(self.stream)
+        self.events.append((kind, s, e))
+        return r
+
+    def totals(self):
+        out = {}
+        for kind, s, e in self.events:
+            n, t = out.get(kind, (0, 0.0))
+            out[kind] = (n + 1, t + s.elapsed_time(e))
+        return out
+
+
+# ---------------------------------------------------------------- workloads
+class LinearWorkload:
+    """One quantized linear: Y = BF16(MXFP8(X) MXFP8(W)^T + b)."""
+
+    def __init__(self, name, M, K, N, seed, desc):
+        self.name, self.M, self.K, self.N, self.seed, self.desc = name, M, K, N, seed, desc
+
+    def config(self):
+        return {"M": self.M, "K": self.K, "N": self.N}
+
+    def flops(self):
+        return 2.0 * self.M * self.N * self.K
+
+    def quant_bytes(self):
+        return self.M * self.K * (2 + 1) + self.M * self.K // 32
+
+    def gemm_bytes(self):
+        M, K, N = self.M, self.K, self.N
+        return M * K * (1 + 1 / 32) + N * K * (1 + 1 / 32) + 2 * M * N + 2 * N
+
+    def setup(self, dev):
+        from mxfp8_w8a8_quantized_b200 import mxfp8, synth
+        self.mx = mxfp8
+        M, K, N, s = self.M, self.K, self.N, self.seed
+        self.x = synth.activations_device(M, K, s, 0, dev)
+        w = synth.weights_device(N, K, s, 0, dev)
+        self.b = synth.bias_device(N, s, 0, dev)
+        self.wq, self.ws = mxfp8.quantize_weight(w)      # offline weight quantization
+        del w
+        self.xq = torch.empty((M, K), dtype=torch.uint8, device=dev)
+        self.xs = torch.empty(mxfp8.scale_bytes(M, K), dtype=torch.uint8, device=dev)
+        self.y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        self.launches = 2
+
+    def step(self, T):
+        mx = self.mx
+        T("quant", mx.quantize, self.x, codes=self.xq, scales=self.xs)
+        T("gemm", mx.gemm_prequant, self.xq, self.xs, self.wq, self.ws, self.b, out=self.y)
+
+    def e2e_io(self):
+        return self.x, self.y
+
+    def e2e_step(self, x_dev, y_dev, ws):
+        self.mx.linear(x_dev, self.wq, self.ws, self.b, out=y_dev, workspace=ws)
+
+    def e2e_workspace(self, dev):
+        return torch.empty(self.mx.linear_workspace_bytes(self.M, self.K), dtype=torch.uint8, device=dev)
+
+
+class FFNPairWorkload(LinearWorkload):
+    """ffn.net.0.proj -> GELU(tanh) -> ffn.net.2 at M tokens."""
+
+    def __init__(self, name, M, seed, desc):
+        from mxfp8_w8a8_quantized_b200 import synth
+        super().__init__(name, M, synth.HIDDEN, synth.FFN, seed, desc)
+
+    def config(self):
+        return {"M": self.M, "hidden": self.K, "ffn": self.N}
+
+    def flops(self):
+        return 2 * 2.0 * self.M * self.N * self.K
+
+    def quant_bytes(self):
+        return self.M * (self.K + self.N) * 3 + self.M * (self.K + self.N) // 32
+
+    def gemm_bytes(self):
+        M, H, F = self.M, self.K, self.N
+        one = M * H * (1 + 1 / 32) + F * H * (1 + 1 / 32) + 2 * M * F + 2 * F
+        two = M * F * (1 + 1 / 32) + H * F * (1 + 1 / 32) + 2 * M * H + 2 * H
+        return one + two
+
+    def setup(self, dev):
+        from mxfp8_w8a8_quantized_b200 import mxfp8, synth
+        from mxfp8_w8a8_quantized_b200.workloads import QLinear, Workspace
+        self.mx = mxfp8
+        M, H, F, s = self.M, self.K, self.N, self.seed
+        self.x = synth.activations_device(M, H, s, 0, dev)
+        self.l0 = QLinear.random(H, F, s, 1, dev)
+        self.l2 = QLinear.random(F, H, s, 2, dev)
+        self.ws_ = Workspace(M * F, M, F, dev)
+        self.f = torch.empty((M, F), dtype=torch.bfloat16, device=dev)
+        self.y = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+        self.launches = 5
+
+    def _run(self, T, x, y):
+        mx = self.mx
+        xq, xs = T("quant", self.ws_.quantize, x)
+        T("gemm", self.l0, xq, xs, out=self.f)
+        T("gelu", mx.gelu_tanh, self.f, out=self.f)
+        fq, fs = T("quant", self.ws_.quantize, self.f)
+        T("gemm", self.l2, fq, fs, out=y)
+
+    def step(self, T):
+        self._run(T, self.x, self.y)
+
+    def e2e_step(self, x_dev, y_dev, ws):
+        self._run(lambda k, f, *a, **kw: f(*a, **kw), x_dev, y_dev)
+
+    def e2e_workspace(self, dev):
+        return None
+
+
+class BlocksWorkload(LinearWorkload):
+    """`nblocks` Wan blocks (10 quantized linears each) at M video / T text tokens."""
+
+    def __init__(self, name, M, T, nblocks, seed, desc):
+        from mxfp8_w8a8_quantized_b200 import synth
+        super().__init__(name, M, synth.HIDDEN, synth.FFN, seed, desc)
+        self.T, self.nblocks = T, nblocks
+
+    def config(self):
+        return {"M": self.M, "text_tokens": self.T, "blocks": self.nblocks, "hidden": self.K, "ffn": self.N}
+
+    def _per_block(self):
+        from mxfp8_w8a8_quantized_b200 import synth
+        fl, qb, gb = 0.0, 0.0, 0.0
+        for _, K, N, kind in synth.block_linears():
+            rows = self.M if kind == "video" else self.T
+            fl += 2.0 * rows * K * N
+            gb += rows * K * (1 + 1 / 32) + N * K * (1 + 1 / 32) + 2 * rows * N + 2 * N
+        # distinct quantizations: x (q/k/v), v1, o1, ctx (k/v), q2, o2, gelu out
+        for rows, K in [(self.M, self.K)] * 5 + [(self.T, self.K), (self.M, self.N)]:
+            qb += rows * K * 3 + rows * K // 32
+        return fl, qb, gb
+
+    def flops(self):
+        return self.nblocks * self._per_block()[0]
+
+    def quant_bytes(self):
+        return self.nblocks * self._per_block()[1]
+
+    def gemm_bytes(self):
+        return self.nblocks * self._per_block()[2]
+
+    def setup(self, dev):
+        from mxfp8_w8a8_quantized_b200 import mxfp8, synth
+        from mxfp8_w8a8_quantized_b200.workloads import Block, workspaces
+        self.mx = mxfp8
+        s = self.seed
+        self.x = synth.activations_device(self.M, self.K, s, 1000, dev)
+        self.ctx = synth.activations_device(self.T, self.K, s, 1001, dev)
+        self.blocks = [Block(s, b, dev) for b in range(self.nblocks)]
+        self.wa, self.wb = workspaces(self.M, self.T, dev)
+        self.y = None
+        self.launches = self.nblocks * (10 + 7 + 1)
+
+    def _run(self, T, x):
+        from mxfp8_w8a8_quantized_b200.workloads import QLinear
+        orig = QLinear.__call__
+        wsq_a, wsq_b = self.wa.quantize, self.wb.quantize
+        try:
+            QLinear.__call__ = lambda lin, xq, xs, out=None: T("gemm", orig, lin, xq, xs, out=out)
+            self.wa.quantize = lambda t: T("quant", wsq_a, t)
+            self.wb.quantize = lambda t: T("quant", wsq_b, t)
+            gelu = self.mx.gelu_tanh
+            self.mx.gelu_tanh = lambda t, out=None: T("gelu", gelu, t, out=out)
+            y = x
+            for blk in self.blocks:
+                y = blk.forward(y, self.ctx, self.wa, self.wb)
+            return y
+        finally:
+            QLinear.__call__ = orig
+            self.wa.quantize, self.wb.quantize = wsq_a, wsq_b
+            self.mx.gelu_tanh = gelu
+
+    def step(self, T):
+        self.y = self._run(T, self.x)
+
+    def e2e_io(self):
+        return self.x, torch.empty_like(self.x)
+
+    def e2e_step(self, x_dev, y_dev, ws):
+        y_dev.copy_(self._run(lambda k, f, *a, **kw: f(*a, **kw), x_dev))
+
+    def e2e_workspace(self, dev):
+        return None
+
+
+def make_workload(name):
+    from mxfp8_w8a8_quantized_b200 import synth
+    H, F = synth.HIDDEN, synth.FFN
+    M1, M2, T = synth.TOKENS_480P, synth.TOKENS_832x1104, synth.TEXT_TOKENS
+    if name == "c0_small":
+        return LinearWorkload(name, 256, 512, 512, 0, "single linear 256x512x512")
+    if name == "c1_q_proj_480p":
+        return LinearWorkload(name, M1, H, H, 1, "Wan2.2 A14B attn1.to_q at 480x832, 81 frames (21x30x52 tokens)")
+    if name == "ffn0_832x1104":
+        return LinearWorkload(name, M2, H, F, 2, "Wan2.2 A14B ffn.net.0.proj at 832x1104, 81 frames")
+    if name == "ffn2_832x1104":
+        return LinearWorkload(name, M2, F, H, 2, "Wan2.2 A14B ffn.net.2 at 832x1104, 81 frames")
+    if name == "c2_ffn_pair_832x1104":
+        return FFNPairWorkload(name, M2, 2, "Wan2.2 A14B FFN pair (5120->13824->5120, GELU-tanh) at 832x1104")
+    if name == "c3_block_832x1104":
+        return BlocksWorkload(name, M2, T, 1, 3, "one Wan2.2 A14B block's 10 quantized linears at 832x1104")
+    if name == "c4_step_832x1104":
+        return BlocksWorkload(name, M2, T, synth.BLOCKS, 4,
+                              "one denoising step: 40 blocks x 10 quantized linears at 832x1104")
+    raise ValueError(name)
+
+
 # ---------------------------------------------------------------- our arm
-def run_ours(args, world, rank, local):
-    from mxfp8_w8a8_quantized_b200 import mxfp8, synth
-
-    shp = workload_shape(args.workload)
-    M, K, N, seed = shp["M"], shp["K"], shp["N"], shp["seed"]
-    dev = torch.device("cuda", local)
-    # synthetic inputs drawn on the device (same recipe as the tests)
-    x = synth.activations_device(M, K, seed, 0, dev)
-    w = synth.weights_device(N, K, seed, 0, dev)
-    b = synth.bias_device(N, seed, 0, dev)
-    wq, ws = mxfp8.quantize_weight(w)          # offline weight quantization
-    del w
-    xq = torch.empty((M, K), dtype=torch.uint8, device=dev)
-    xs = torch.empty(mxfp8.scale_bytes(M, K), dtype=torch.uint8, device=dev)
-    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+def run_ours(args, ranks, dev):
+    wl = make_workload(args.workload)
+    wl.setup(dev)
     stream = torch.cuda.current_stream(dev)
-
-    def step():
-        mxfp8.quantize(x, codes=xq, scales=xs)
-        mxfp8.gemm_prequant(xq, xs, wq, ws, b, out=y)
-
+    mx = wl.mx
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    T = KernelTimer(stream)
     for _ in range(max(args.warmup, 3)):
         flush.zero_()
-        step()
+        wl.step(T)
     torch.cuda.synchronize()
-    if mxfp8.device_status() != 0:
+    if mx.device_status() != 0:
         raise RuntimeError("kernel reported a pipeline timeout during warm-up")
 
-    K_steps = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K_steps)]
-    barrier(world)
+    steps = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    T.on = True
+    ranks.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        for i in range(K_steps):
+    with ClockSampler(dev.index or 0) as clk:
+        for i in range(steps):
             flush.zero_()                      # L2 flushed between timed steps
-            e0, e1, e2 = ev[i]
-            e0.record(stream)
-            mxfp8.quantize(x, codes=xq, scales=xs)
-            e1.record(stream)
-            mxfp8.gemm_prequant(xq, xs, wq, ws, b, out=y)
-            e2.record(stream)
+            ev[i][0].record(stream)
+            wl.step(T)
+            ev[i][1].record(stream)
         torch.cuda.synchronize()
-    barrier(world)
-    if mxfp8.device_status() != 0:
+    ranks.barrier()
+    if mx.device_status() != 0:
         raise RuntimeError("kernel reported a pipeline timeout")
-    q_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    g_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    s_ms = [e[0].elapsed_time(e[2]) for e in ev]
-    total_ms = max_over_ranks(world, sum(s_ms))
-    ms_per_step = total_ms / K_steps
-    flops = 2.0 * M * N * K
-    value = world * flops * K_steps / (total_ms * 1e-3) / 1e12
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = ranks.max(sum(step_ms))
+    ms_per_step = total_ms / steps
+    value = ranks.world * wl.flops() * steps / (total_ms * 1e-3) / 1e12
 
     hbm, bf16, peak_src = load_peaks()
     fp8_peak = bf16 * FP8_OVER_BF16
-    gemm_ms = statistics.mean(g_ms)
-    quant_ms = statistics.mean(q_ms)
-    gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
-    quant_bytes = M * K * 2 + M * K + M * K // 32
-    quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
-    traffic = load_traffic(args.workload)
-
+    tot = T.totals()
+    g_n, g_ms = tot["gemm"]
+    q_n, q_ms = tot["quant"]
+    gemm_tflops = wl.flops() * steps / (g_ms * 1e-3) / 1e12
+    quant_gbs = wl.quant_bytes() * steps / (q_ms * 1e-3) / 1e9
     out = {
         "metric": METRIC,
         "value": round(value, 2),
         "unit": "TFLOP/s",
-        "n_gpus": world,
-        "steps": K_steps,
+        "n_gpus": ranks.world,
+        "steps": steps,
         "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True,
@@ -242,64 +442,71 @@ def run_ours(args, world, rank, local):
         "dtype": "e4m3 (MXFP8 operands, fp32 accumulate, bf16 out)",
         "data": "synthetic (seeded N(0,1) activations with 1% x20 outlier channels, N(0,1/sqrt(K)) weights, "
                 "N(0,0.01) f16 bias)",
-        "config": {"workload": args.workload, "desc": shp["desc"], "M": M, "K": K, "N": N,
-                   "l2": "flushed between timed steps (256 MiB write outside the step events)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "config": dict(workload=wl.name, desc=wl.desc, **wl.config(),
+                       l2="flushed between timed steps (256 MiB write outside the step events)",
+                       parallelism=f"replicas x{ranks.world}" if ranks.world > 1 else "single GPU"),
         "roofline": {"bound": "tensor", "kernel": "mxfp8_gemm_kernel",
                      "achieved": round(gemm_tflops, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
                      "frac": round(gemm_tflops / fp8_peak, 4),
                      "peak_source": f"{peak_src} bf16 burst x {FP8_OVER_BF16} (nominal FP8/BF16 ratio)",
-                     "traffic": traffic,
-                     "algorithmic_bytes": M * K * (1 + 1 / 32) + N * K * (1 + 1 / 32) + 2 * M * N + 2 * N,
-                     "avg_launch_ms": round(gemm_ms, 4)},
+                     "traffic": load_traffic(wl.name),
+                     "algorithmic_bytes_per_step": round(wl.gemm_bytes()),
+                     "launches_per_step": g_n // steps, "avg_launch_ms": round(g_ms / g_n, 4)},
         "quant": {"kernel": "mx_quantize_kernel", "achieved_gbs": round(quant_gbs, 1), "peak_gbs": hbm,
                   "frac": round(quant_gbs / hbm, 4), "peak_source": f"{peak_src} copy",
-                  "bytes_per_launch": quant_bytes, "avg_launch_ms": round(quant_ms, 4)},
-        "gpu_launches": 2 * K_steps,
+                  "bytes_per_step": wl.quant_bytes(), "launches_per_step": q_n // steps,
+                  "avg_launch_ms": round(q_ms / q_n, 4)},
+        "gpu_launches": wl.launches * steps,
         "clocks": clk.summary(),
     }
+    if "gelu" in tot:
+        n, ms = tot["gelu"]
+        out["gelu"] = {"launches_per_step": n // steps, "avg_launch_ms": round(ms / n, 4)}
     if not args.no_e2e:
-        out["e2e"] = run_e2e(args, mxfp8, x, wq, ws, b, M, K, N, world, dev)
+        out["e2e"] = run_e2e(args, wl, ranks, dev)
     return out
 
 
-def run_e2e(args, mxfp8, x_dev, wq, ws, b, M, K, N, world, dev):
+def run_e2e(args, wl, ranks, dev):
     """Same metric through the public API with host buffers: pinned host X ->
-    device, mxfp8.linear, Y -> pinned host, all inside the timed region."""
-    x_host = torch.empty((M, K), dtype=torch.bfloat16, pin_memory=True)
+    device, the workload, Y -> pinned host, all inside the timed region."""
+    x_dev, y_ref = wl.e2e_io()
+    x_host = torch.empty(x_dev.shape, dtype=x_dev.dtype, pin_memory=True)
     x_host.copy_(x_dev.cpu())
-    y_host = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
+    y_host = torch.empty(y_ref.shape, dtype=y_ref.dtype, pin_memory=True)
     x_stage = torch.empty_like(x_dev)
-    y_dev = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    ws_buf = torch.empty(mxfp8.linear_workspace_bytes(M, K), dtype=torch.uint8, device=dev)
+    y_dev = torch.empty_like(y_ref)
+    ws = wl.e2e_workspace(dev)
     stream = torch.cuda.current_stream(dev)
-    steps = max(3, min(args.steps, 20))
+    steps = max(3, min(args.steps, 20 if wl.flops() < 1e14 else 3))
 
     def step():
         x_stage.copy_(x_host, non_blocking=True)
-        mxfp8.linear(x_stage, wq, ws, b, out=y_dev, workspace=ws_buf)
+        wl.e2e_step(x_stage, y_dev, ws)
         y_host.copy_(y_dev, non_blocking=True)
 
-    for _ in range(3):
+    for _ in range(2):
         step()
     torch.cuda.synchronize()
-    barrier(world)
+    ranks.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(steps):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = max_over_ranks(world, e0.elapsed_time(e1))
-    barrier(world)
-    value = world * 2.0 * M * N * K * steps / (ms * 1e-3) / 1e12
-    return {"value": round(value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": M * K * 2,
-            "d2h_bytes_per_step": M * N * 2, "steps": steps, "ms_per_step": round(ms / steps, 3)}
+    ms = ranks.max(e0.elapsed_time(e1))
+    ranks.barrier()
+    value = ranks.world * wl.flops() * steps / (ms * 1e-3) / 1e12
+    return {"value": round(value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+            "d2h_bytes_per_step": y_host.numel() * y_host.element_size(), "steps": steps,
+            "ms_per_step": round(ms / steps, 3)}
 
 
 def load_traffic(workload):
-    """dram bytes per GEMM launch from the committed ncu summary, if it is for
-    the current kernel build (profiles/<kernel>_<workload>.json)."""
+    """DRAM bytes per GEMM launch from the committed ncu summary
+    (profiles/mxfp8_gemm_<workload>.json), if it was taken on the current
+    kernel sources; else None."""
     path = os.path.join(ROOT, "profiles", f"mxfp8_gemm_{workload}.json")
     try:
         d = json.load(open(path))
@@ -312,17 +519,17 @@ def load_traffic(workload):
 
 
 # ---------------------------------------------------------------- CPU oracle
-def oracle_sample(shp, rows, seed_rows=0):
-    """Inputs of a bounded sample: `rows` rows of X and all of W (quantized
-    by the oracle outside the timed region, as the weights are offline)."""
+def oracle_sample(wl, rows):
+    """A bounded sample of a single-linear workload for the oracle: `rows`
+    rows of X and all of W (quantized by the oracle outside the timed region,
+    as weights are offline)."""
     import numpy as np
 
     import oracle
     from mxfp8_w8a8_quantized_b200 import synth
-    M, K, N, seed = shp["M"], shp["K"], shp["N"], shp["seed"]
-    x = synth.activations(rows, K, seed, index=100 + seed_rows)
-    w = synth.weights(N, K, seed, index=100)
-    b = synth.bias(N, seed, index=100)
+    x = synth.activations(rows, wl.K, wl.seed, index=100)
+    w = synth.weights(wl.N, wl.K, wl.seed, index=100)
+    b = synth.bias(wl.N, wl.seed, index=100)
     wq, ws = oracle.quantize_f32(w.numpy())
     xb = x.view(torch.int16).numpy().view(np.uint16)
     bb = b.view(torch.int16).numpy().view(np.uint16)
@@ -330,58 +537,71 @@ def oracle_sample(shp, rows, seed_rows=0):
 
 
 def oracle_step(xb, wq, ws, bb):
+    """One step of the oracle on the sample: quantize the rows, FP64 linear."""
     import oracle
     xq, xs = oracle.quantize_bf16(xb)
     return oracle.linear(xq, xs, wq, ws, bb)
 
 
-def cpu_baseline(shp, target_s):
+def size_sample(wl, target_s, max_rows=None):
+    """Rows whose oracle step takes about target_s seconds."""
+    rows, dt = 4, 0.0
+    for _ in range(6):
+        xb, wq, ws, bb = oracle_sample(wl, rows)
+        t0 = time.perf_counter()
+        oracle_step(xb, wq, ws, bb)
+        dt = time.perf_counter() - t0
+        if dt >= 0.5 * target_s:
+            break
+        rows = int(min(wl.M, max(rows * 2, rows * 0.9 * target_s / max(dt, 1e-3))))
+        if max_rows:
+            rows = min(rows, max_rows)
+    return rows
+
+
+def cpu_baseline(wl, target_s):
     import oracle
-    K, N = shp["K"], shp["N"]
-    xb, wq, ws, bb = oracle_sample(shp, 2)
-    t0 = time.perf_counter()
-    oracle_step(xb, wq, ws, bb)
-    t_probe = (time.perf_counter() - t0) / 2
-    rows = int(max(1, min(shp["M"], target_s / max(t_probe, 1e-6))))
-    xb, wq, ws, bb = oracle_sample(shp, rows)
+    if not isinstance(wl, LinearWorkload) or type(wl) is not LinearWorkload:
+        return {"value": None, "unit": "TFLOP/s", "kind": "oracle", "cores": oracle.num_threads(),
+                "sample": "not measured for chained workloads"}
+    rows = size_sample(wl, target_s)
+    xb, wq, ws, bb = oracle_sample(wl, rows)
     t0 = time.perf_counter()
     oracle_step(xb, wq, ws, bb)
     dt = time.perf_counter() - t0
-    return {"value": round(2.0 * rows * N * K / dt / 1e12, 6), "unit": "TFLOP/s",
+    return {"value": round(2.0 * rows * wl.N * wl.K / dt / 1e12, 6), "unit": "TFLOP/s",
             "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{rows} of {shp['M']} rows (quantize + FP64 linear over all {N} columns, K={K}); "
+            "sample": f"{rows} of {wl.M} rows (quantize + FP64 linear over all {wl.N} columns, K={wl.K}); "
                       f"weights quantized outside the timed region; {dt:.1f} s"}
 
 
-def run_reference(args, world, rank):
+def run_reference(args, ranks):
     """The oracle as the reference arm: CPU, rank 0 only."""
     import oracle
-    shp = workload_shape(args.workload)
-    M, K, N = shp["M"], shp["K"], shp["N"]
-    if rank != 0:
+    wl = make_workload(args.workload)
+    if type(wl) is not LinearWorkload:
+        wl = make_workload("c1_q_proj_480p") if args.workload == "c1_q_proj_480p" else \
+            LinearWorkload(wl.name, wl.M, wl.K, wl.K, wl.seed, wl.desc + " (first linear only)")
+    if ranks.rank != 0:
         return None
-    budget = 150.0  # seconds for warm-up + timed steps together
-    xb, wq, ws, bb = oracle_sample(shp, 1)
-    t0 = time.perf_counter()
-    oracle_step(xb, wq, ws, bb)
-    t_row = time.perf_counter() - t0
+    budget = args.reference_seconds  # warm-up + timed steps together
     n_steps = args.steps + args.warmup
-    rows = int(max(1, min(M, budget / n_steps / max(t_row, 1e-6))))
-    xb, wq, ws, bb = oracle_sample(shp, rows)
+    rows = size_sample(wl, budget / n_steps)
+    xb, wq, ws, bb = oracle_sample(wl, rows)
     for _ in range(args.warmup):
         oracle_step(xb, wq, ws, bb)
     t0 = time.perf_counter()
     for _ in range(args.steps):
         oracle_step(xb, wq, ws, bb)
     dt = time.perf_counter() - t0
-    value = 2.0 * rows * N * K * args.steps / dt / 1e12
-    sample = f"{rows} of {M} rows per step (quantize + FP64 linear over all {N} columns, K={K})"
+    value = 2.0 * rows * wl.N * wl.K * args.steps / dt / 1e12
+    sample = f"{rows} of {wl.M} rows per step (quantize + FP64 linear over all {wl.N} columns, K={wl.K})"
     return {
         "impl": "reference",
         "metric": METRIC,
         "value": round(value, 6),
         "unit": "TFLOP/s",
-        "n_gpus": world,
+        "n_gpus": ranks.world,
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(dt / args.steps * 1e3, 3),
@@ -390,33 +610,33 @@ def run_reference(args, world, rank):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (same recipe as the GPU arm)",
-        "config": {"workload": args.workload, "desc": shp["desc"], "M": M, "K": K, "N": N},
+        "config": dict(workload=wl.name, desc=wl.desc, **wl.config()),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 
-def main():
-    args = parse()
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
+def main(argv=None):
+    args = parse(argv)
     if args.impl == "reference":
-        out = run_reference(args, world, rank)
+        # CPU only: rank 0 runs the oracle and prints; other ranks exit at once
+        out = run_reference(args, Ranks())
         if out is not None:
             print(json.dumps(out), flush=True)
         return
-    world, rank, local = dist_setup(args.gpus)
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ranks = Ranks(backend="nccl", device=dev)
     try:
-        out = run_ours(args, world, rank, local)
-        if rank == 0:
-            if world == 1 and not args.no_cpu_baseline:
-                out["cpu_baseline"] = cpu_baseline(workload_shape(args.workload), args.cpu_seconds)
+        out = run_ours(args, ranks, dev)
+        if ranks.rank == 0:
+            if ranks.world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = cpu_baseline(make_workload(args.workload), args.cpu_seconds)
             print(json.dumps(out), flush=True)
     finally:
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
+        ranks.close()
 
 
 if __name__ == "__main__":

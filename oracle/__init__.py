@@ -48,6 +48,7 @@ def lib():
         L.orc_quantize_f32.argtypes = [P, I64, I64, P, P]
         L.orc_dequantize.argtypes = [P, P, I64, I64, P]
         L.orc_linear.argtypes = [P, P, I64, I64, P, P, I64, P, P, I64, P, I64, P]
+        L.orc_linear_f32acc.argtypes = [P, P, I64, I64, P, P, I64, P, P, I64, P, I64, P]
         L.orc_bf16_rne_array.argtypes = [P, I64, P]
         L.orc_gelu_tanh_bf16.argtypes = [P, I64, P]
         L.orc_num_threads.restype = ctypes.c_int
@@ -179,6 +180,26 @@ def linear(xq, xs, wq, ws, bias_bits=None, rows=None, cols=None):
     Y = np.empty((nr, nc), dtype=np.float64)
     lib().orc_linear(_ptr(xq), _ptr(xs), M, K, _ptr(wq), _ptr(ws), N, _ptr(b),
                      _ptr(r), nr, _ptr(c), nc, _ptr(Y))
+    return Y
+
+
+def linear_f32acc(xq, xs, wq, ws, bias_bits=None, rows=None, cols=None):
+    """As `linear`, but accumulated in FP32 in increasing k (one admissible
+    FP32 evaluation order); returns the FP32 results as float64."""
+    xq = _c(xq, np.uint8)
+    xs = _c(xs, np.uint8)
+    wq = _c(wq, np.uint8)
+    ws = _c(ws, np.uint8)
+    M, K = xq.shape
+    N = wq.shape[0]
+    r = None if rows is None else _c(rows, np.int64)
+    c = None if cols is None else _c(cols, np.int64)
+    nr = M if r is None else r.size
+    nc = N if c is None else c.size
+    b = None if bias_bits is None else _c(bias_bits, np.uint16)
+    Y = np.empty((nr, nc), dtype=np.float64)
+    lib().orc_linear_f32acc(_ptr(xq), _ptr(xs), M, K, _ptr(wq), _ptr(ws), N, _ptr(b),
+                            _ptr(r), nr, _ptr(c), nc, _ptr(Y))
     return Y
 
 

@@ -319,6 +319,52 @@ void orc_linear(const uint8_t *xq, const uint8_t *xs, int64_t M, int64_t K,
     free(wd);
 }
 
+/*
+ * The same linear layer with FP32 accumulation in increasing k (one FP32
+ * rounding per addition, then the F16 bias added in FP32): one admissible
+ * evaluation order of the layer's FP32 accumulation.  Each product of two
+ * E4M3 values and two powers of two is exact in FP32 for the scale ranges
+ * of real data.  Used to measure how far two valid evaluations of a chain of
+ * layers drift apart.
+ */
+void orc_linear_f32acc(const uint8_t *xq, const uint8_t *xs, int64_t M, int64_t K,
+                       const uint8_t *wq, const uint8_t *ws, int64_t N, const uint16_t *bias,
+                       const int64_t *rows, int64_t nr, const int64_t *cols, int64_t nc, double *Y)
+{
+    (void)M;
+    (void)N;
+    int64_t nb = K / 32;
+    double *wd = (double *)malloc((size_t)nc * (size_t)K * sizeof(double));
+    if (!wd)
+        return;
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < nc; ++j) {
+        int64_t n = cols ? cols[j] : j;
+        for (int64_t k = 0; k < K; ++k)
+            wd[j * K + k] = orc_e4m3_decode(wq[n * K + k]) * orc_e8m0_decode(ws[n * nb + k / 32]);
+    }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < nr; ++i) {
+        int64_t r = rows ? rows[i] : i;
+        double *xd = (double *)malloc((size_t)K * sizeof(double));
+        if (!xd)
+            continue;
+        for (int64_t k = 0; k < K; ++k)
+            xd[k] = orc_e4m3_decode(xq[r * K + k]) * orc_e8m0_decode(xs[r * nb + k / 32]);
+        for (int64_t j = 0; j < nc; ++j) {
+            int64_t n = cols ? cols[j] : j;
+            float acc = 0.0f;
+            for (int64_t k = 0; k < K; ++k)
+                acc = acc + (float)(xd[k] * wd[j * K + k]);
+            if (bias)
+                acc = acc + (float)orc_f16_decode(bias[n]);
+            Y[i * nc + j] = (double)acc;
+        }
+        free(xd);
+    }
+    free(wd);
+}
+
 /* FP64 values -> BF16 bits (RNE), elementwise. */
 void orc_bf16_rne_array(const double *v, int64_t n, uint16_t *out)
 {

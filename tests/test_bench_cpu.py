@@ -1,0 +1,86 @@
+"""Host-side logic of bench.py without a GPU: the rank helpers over a
+world_size-2 gloo group (barrier, max over ranks -- the only collectives the
+replicas use), and the reference arm (the CPU oracle), including its
+behaviour under torchrun where only rank 0 works and prints."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import bench
+    r = bench.Ranks(backend="gloo")
+    r.barrier()
+    m = r.max(10.0 + 5.0 * rank)          # the slowest rank's time wins
+    r.barrier()
+    r.close()
+    q.put((rank, m))
+
+
+def test_ranks_barrier_and_max_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ps = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in ps:
+        p.start()
+    for p in ps:
+        p.join(120)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=10) for _ in range(2))
+    assert got == [(0, 15.0), (1, 15.0)]
+
+
+def _bench(args, env):
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py")] + args, cwd=ROOT,
+                          env=dict(os.environ, **env), capture_output=True, text=True, timeout=600)
+
+
+def test_reference_arm_prints_one_json_line():
+    r = _bench(["--impl", "reference", "--workload", "c0_small", "--steps", "2", "--warmup", "1",
+                "--reference-seconds", "3"], {})
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["config"]["workload"] == "c0_small"
+
+
+def test_reference_arm_nonzero_rank_exits_without_work():
+    r = _bench(["--impl", "reference", "--workload", "c0_small", "--steps", "2", "--warmup", "1",
+                "--reference-seconds", "3"], {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip() == ""
+
+
+def test_workload_accounting():
+    sys.path.insert(0, ROOT)
+    import bench
+    c1 = bench.make_workload("c1_q_proj_480p")
+    assert c1.flops() == 2.0 * 32760 * 5120 * 5120
+    blk = bench.make_workload("c3_block_832x1104")
+    step = bench.make_workload("c4_step_832x1104")
+    # 8 hidden x hidden linears (two on 512 text tokens) + the FFN pair
+    expect = 2.0 * (6 * 75348 * 5120 * 5120 + 2 * 512 * 5120 * 5120 + 2 * 75348 * 5120 * 13824)
+    assert blk.flops() == pytest.approx(expect)
+    assert step.flops() == pytest.approx(40 * expect)

@@ -1,0 +1,224 @@
+"""GPU parity at the full sizes of the five Wan workloads.
+
+* Single linears (the Q projection at 480x832; ffn.net.0.proj and ffn.net.2
+  at 832x1104; the first linears of a block): codes and scales bit-exact
+  against the oracle, Y within |Y - Yref| <= 2^-7 |Yref| + 1e-3 rms(Yref) on
+  sampled rows x columns (the ragged last tile and tile edges included).
+* Chains (FFN pair, one block, a 40-block step): every linear's BF16 output is
+  one of several correct roundings (the FP32 accumulation order is not
+  fixed), and a later linear re-quantizes it, so any two admissible
+  evaluations of a chain drift apart.  The exact oracle chain (FP64 sums) is
+  the reference; a second admissible evaluation -- the oracle with FP32
+  accumulation in increasing k -- gives the drift two valid evaluations
+  show on the same rows (D_ref).  The GPU chain's drift from the exact chain
+  (D_gpu, per-row relative L2) must stay within that band:
+      mean D_gpu <= 2 mean D_ref + 2e-3
+      max  D_gpu <= 2 max  D_ref + 3e-2     (oracle_chain.chain_band)
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import assert_within_tol, bf16_bits, bf16_values, f16_bits, unswizzle
+from mxfp8_w8a8_quantized_b200 import synth
+from oracle_chain import OracleLinear, block_rows, chain_band
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+def check_chain(name, got, ref64, ref32):
+    ok, stats = chain_band(got, ref64, ref32)
+    record(name, **stats)
+    assert ok, (name, stats)
+
+
+OUT = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "gpurun_out")
+
+
+def record(name, **kv):
+    """Keep the observed chain distances next to the run's other outputs."""
+    try:
+        os.makedirs(OUT, exist_ok=True)
+        with open(os.path.join(OUT, "chain_parity.jsonl"), "a") as f:
+            f.write(json.dumps(dict(test=name, **kv)) + "\n")
+    except OSError:
+        pass
+
+
+@pytest.fixture(scope="module")
+def mx():
+    from mxfp8_w8a8_quantized_b200 import mxfp8
+    return mxfp8
+
+
+DEV = "cuda"
+
+
+def sample_rows(M, n=192, seed=0):
+    rng = np.random.default_rng(seed)
+    edge = [0, 1, 127, 128, 255, 256, M // 2, M - 129, M - 128]
+    tail = list(range(max(0, M - 64), M))              # the ragged last tile
+    rest = rng.choice(M, n, replace=False)
+    return np.unique(np.clip(np.array(edge + tail + list(rest)), 0, M - 1))
+
+
+def sample_cols(N, n=160, seed=1):
+    rng = np.random.default_rng(seed)
+    edge = [0, 7, 8, 31, 32, 255, 256, N - 256, N - 1]
+    return np.unique(np.clip(np.array(edge + list(rng.choice(N, n, replace=False))), 0, N - 1))
+
+
+def host_weights(N, K, seed, index):
+    w = synth.weights_device(N, K, seed, index, DEV).cpu().numpy()
+    b = f16_bits(synth.bias_device(N, seed, index, DEV))
+    return w, b
+
+
+def check_linear(mx, x, w, b, rows, cols, what, all_codes=False):
+    """x, w, b on the GPU; checks codes/scales and sampled Y of one linear."""
+    M, K = x.shape
+    N = w.shape[0]
+    wq, ws = mx.quantize_weight(w)
+    xq, xs = mx.quantize(x)
+    y = mx.gemm_prequant(xq, xs, wq, ws, b)
+    y_lin = mx.linear(x, wq, ws, b)
+    torch.cuda.synchronize()
+    assert mx.device_status() == 0
+    assert torch.equal(y, y_lin), f"{what}: mxfp8_linear differs from quantize + gemm_prequant"
+    rows_t = torch.from_numpy(rows).to(DEV)
+    x_rows = bf16_bits(x[rows_t])
+    oq, os_ = oracle.quantize_f32(w.cpu().numpy())
+    assert np.array_equal(wq.cpu().numpy(), oq), f"{what}: weight codes"
+    assert np.array_equal(unswizzle(ws.cpu().numpy(), N, K), os_), f"{what}: weight scales"
+    if all_codes:
+        rq, rs = oracle.quantize_bf16(bf16_bits(x))
+        assert np.array_equal(xq.cpu().numpy(), rq), f"{what}: activation codes"
+        assert np.array_equal(unswizzle(xs.cpu().numpy(), M, K), rs), f"{what}: activation scales"
+        rq, rs = rq[rows], rs[rows]
+    else:
+        rq, rs = oracle.quantize_bf16(x_rows)
+        assert np.array_equal(xq[rows_t].cpu().numpy(), rq), f"{what}: activation codes (sampled rows)"
+        assert np.array_equal(unswizzle(xs.cpu().numpy(), M, K)[rows], rs), f"{what}: activation scales"
+    yref = oracle.linear(rq, rs, oq, os_, f16_bits(b), cols=cols)
+    ysub_bits = bf16_bits(y[rows_t][:, torch.from_numpy(cols).to(DEV)])
+    assert_within_tol(bf16_values(ysub_bits), yref, what)
+    # how often the BF16 output differs from the rounded exact result, for the
+    # GPU and for the FP32-in-k-order evaluation (both are admissible)
+    exact_bits = oracle.bf16_rne(yref)
+    f32_bits = oracle.bf16_rne(oracle.linear_f32acc(rq, rs, oq, os_, f16_bits(b), cols=cols))
+    record("bf16_flips_" + what.replace(" ", "_"), gpu=float((ysub_bits != exact_bits).mean()),
+           f32_in_order=float((f32_bits != exact_bits).mean()), outputs=int(exact_bits.size))
+    return y
+
+
+def test_q_projection_480p_full_size(mx):
+    """M = 32760 (21x30x52 tokens), K = N = 5120: all codes and scales
+    bit-exact, sampled Y within tolerance."""
+    M, K, N, seed = synth.TOKENS_480P, synth.HIDDEN, synth.HIDDEN, 1
+    x = synth.activations_device(M, K, seed, 0, DEV)
+    w = synth.weights_device(N, K, seed, 0, DEV)
+    b = synth.bias_device(N, seed, 0, DEV)
+    check_linear(mx, x, w, b, sample_rows(M), sample_cols(N), "Q projection", all_codes=True)
+
+
+def test_ffn_pair_832x1104_full_size(mx):
+    """ffn.net.0.proj (75348 x 5120 -> 13824) and ffn.net.2 (75348 x 13824 ->
+    5120), each on generator inputs of its exact shape; then the chained pair
+    (GELU between) against the oracle's chain on sampled rows."""
+    M, H, F, seed = synth.TOKENS_832x1104, synth.HIDDEN, synth.FFN, 2
+    rows = sample_rows(M)
+    x = synth.activations_device(M, H, seed, 0, DEV)
+    w0 = synth.weights_device(F, H, seed, 1, DEV)
+    b0 = synth.bias_device(F, seed, 1, DEV)
+    f = check_linear(mx, x, w0, b0, rows, sample_cols(F), "ffn.net.0.proj", all_codes=True)
+    w2 = synth.weights_device(H, F, seed, 2, DEV)
+    b2 = synth.bias_device(H, seed, 2, DEV)
+    h = synth.activations_device(M, F, seed, 3, DEV)
+    check_linear(mx, h, w2, b2, rows, sample_cols(H), "ffn.net.2")
+    del h
+    torch.cuda.empty_cache()
+
+    # the chain: f -> GELU (in place) -> ffn.net.2
+    wq2, ws2 = mx.quantize_weight(w2)
+    mx.gelu_tanh(f, out=f)
+    y = mx.linear(f, wq2, ws2, b2)
+    torch.cuda.synchronize()
+    crow = rows[:: max(1, len(rows) // 24)]
+    x_rows = bf16_bits(x[torch.from_numpy(crow).to(DEV)])
+    lin0 = OracleLinear(w0.cpu().numpy(), f16_bits(b0))
+    lin2 = OracleLinear(w2.cpu().numpy(), f16_bits(b2))
+    ref64 = bf16_values(lin2(oracle.gelu_tanh_bf16(lin0(x_rows))))
+    ref32 = bf16_values(lin2(oracle.gelu_tanh_bf16(lin0(x_rows, True)), True))
+    got = bf16_values(bf16_bits(y[torch.from_numpy(crow).to(DEV)]))
+    check_chain("ffn_pair_chain", got, ref64, ref32)
+
+
+def test_block_832x1104_full_size(mx):
+    """One block's ten linears at M = 75348 video / 512 text tokens."""
+    from mxfp8_w8a8_quantized_b200.workloads import Block, workspaces
+    M, T, seed = synth.TOKENS_832x1104, synth.TEXT_TOKENS, 3
+    x = synth.activations_device(M, synth.HIDDEN, seed, 1000, DEV)
+    ctx = synth.activations_device(T, synth.HIDDEN, seed, 1001, DEV)
+    blk = Block(seed, 0, DEV)
+    wa, wb = workspaces(M, T, DEV)
+    y, mid = blk.forward(x, ctx, wa, wb, keep=True)
+    torch.cuda.synchronize()
+    assert mx.device_status() == 0
+
+    names = [n for n, _, _, _ in synth.block_linears()]
+    lin = {}
+    for i, (name, K, N, _) in enumerate(synth.block_linears()):
+        if name in ("attn1.to_q", "attn1.to_k"):
+            continue                                   # checked below / not on the chain
+        w, b = host_weights(N, K, seed, i)
+        lin[name] = OracleLinear(w, b)
+    rows = sample_rows(M)
+    cols = sample_cols(synth.HIDDEN)
+    rows_t = torch.from_numpy(rows).to(DEV)
+    cols_t = torch.from_numpy(cols).to(DEV)
+    # first linear: generator input, single-linear tolerance
+    wq1, bq1 = host_weights(synth.HIDDEN, synth.HIDDEN, seed, names.index("attn1.to_q"))
+    q1ref = OracleLinear(wq1, bq1).exact(bf16_bits(x[rows_t]))[:, cols]
+    assert_within_tol(bf16_values(bf16_bits(mid["q1"][rows_t][:, cols_t])), q1ref, "attn1.to_q")
+    # text branch: generator input, all 512 rows
+    k2ref = lin["attn2.to_k"].exact(bf16_bits(ctx))[:, cols]
+    assert_within_tol(bf16_values(bf16_bits(mid["k2"][:, cols_t])), k2ref, "attn2.to_k")
+    # the chain to y
+    crow = rows[:: max(1, len(rows) // 24)]
+    xr = bf16_bits(x[torch.from_numpy(crow).to(DEV)])
+    ref64 = bf16_values(block_rows(xr, lin))
+    ref32 = bf16_values(block_rows(xr, lin, f32acc=True))
+    got = bf16_values(bf16_bits(y[torch.from_numpy(crow).to(DEV)]))
+    check_chain("block_chain", got, ref64, ref32)
+
+
+def test_step_40_blocks_832x1104_full_size(mx):
+    """A denoising step's 400 linears (40 blocks) at full size, block by
+    block; sampled rows of the step's output against the oracle's chain."""
+    from mxfp8_w8a8_quantized_b200.workloads import Block, workspaces
+    M, T, seed, nblocks = synth.TOKENS_832x1104, synth.TEXT_TOKENS, 4, synth.BLOCKS
+    x = synth.activations_device(M, synth.HIDDEN, seed, 1000, DEV)
+    ctx = synth.activations_device(T, synth.HIDDEN, seed, 1001, DEV)
+    crow = sample_rows(M)[::12]
+    crow_t = torch.from_numpy(crow).to(DEV)
+    orc = bf16_bits(x[crow_t])
+    orc32 = orc
+    wa, wb = workspaces(M, T, DEV)
+    chain = ["attn1.to_v", "attn1.to_out", "attn2.to_q", "attn2.to_out", "ffn.net.0.proj", "ffn.net.2"]
+    for blk_i in range(nblocks):
+        blk = Block(seed, blk_i, DEV)
+        x = blk.forward(x, ctx, wa, wb)
+        del blk
+        lin = {}
+        for i, (name, K, N, _) in enumerate(synth.block_linears()):
+            if name in chain:
+                w, b = host_weights(N, K, seed, 10 * blk_i + i)
+                lin[name] = OracleLinear(w, b)
+        orc = block_rows(orc, lin)
+        orc32 = block_rows(orc32, lin, f32acc=True)
+    torch.cuda.synchronize()
+    assert mx.device_status() == 0
+    check_chain("step_chain", bf16_values(bf16_bits(x[crow_t])), bf16_values(orc), bf16_values(orc32))

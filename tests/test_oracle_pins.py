@@ -383,3 +383,46 @@ def test_weight_bytes_match_model_card_order_of_magnitude():
     assert abs(gib - 13.99) / 13.99 < 0.05, gib
     # 2-byte or 4-bit storage would miss by far
     assert abs(2 * elems / 2 ** 30 - 13.99) / 13.99 > 0.5
+
+
+# ------------------------------------------------------------------ FP32 order
+def test_linear_f32acc_is_sequential_float32_sum():
+    # the FP32 evaluation is a left-to-right float32 accumulation of the exact
+    # products: numpy's float32 add.accumulate computes the same sequence
+    rng = np.random.default_rng(41)
+    M, N, K = 3, 4, 96
+    xq = rng.choice(FINITE_CODES, (M, K)).astype(np.uint8)
+    wq = rng.choice(FINITE_CODES, (N, K)).astype(np.uint8)
+    xs = rng.integers(118, 136, (M, K // 32)).astype(np.uint8)
+    ws = rng.integers(118, 136, (N, K // 32)).astype(np.uint8)
+    bias = (rng.standard_normal(N)).astype(np.float16)
+    xd, wd = _torch_dequant(xq, xs), _torch_dequant(wq, ws)
+    got = oracle.linear_f32acc(xq, xs, wq, ws, bias.view(np.uint16))
+    for i in range(M):
+        for j in range(N):
+            prods = (xd[i] * wd[j]).astype(np.float32)
+            assert np.array_equal(prods.astype(np.float64), xd[i] * wd[j])   # products exact
+            s = np.add.accumulate(prods, dtype=np.float32)[-1]
+            s = np.float32(s + np.float32(bias[j]))
+            assert got[i, j] == float(s)
+
+
+def test_linear_f32acc_within_float32_summation_bound():
+    rng = np.random.default_rng(42)
+    M, N, K = 4, 5, 512
+    xq = rng.choice(FINITE_CODES, (M, K)).astype(np.uint8)
+    wq = rng.choice(FINITE_CODES, (N, K)).astype(np.uint8)
+    xs = rng.integers(115, 135, (M, K // 32)).astype(np.uint8)
+    ws = rng.integers(115, 135, (N, K // 32)).astype(np.uint8)
+    f64 = oracle.linear(xq, xs, wq, ws)
+    f32 = oracle.linear_f32acc(xq, xs, wq, ws)
+    absum = np.abs(_torch_dequant(xq, xs)) @ np.abs(_torch_dequant(wq, ws)).T
+    assert (np.abs(f32 - f64) <= K * 2.0 ** -24 * absum).all()
+    # integer-valued cases are exact in both
+    ints = [c for c in range(256) if (c & 0x7F) != 0x7F and float(torch_e4m3_decode([c])[0]).is_integer()
+            and abs(torch_e4m3_decode([c])[0]) <= 16]
+    xq = rng.choice(ints, (M, K)).astype(np.uint8)
+    wq = rng.choice(ints, (N, K)).astype(np.uint8)
+    one = np.full((M, K // 32), 127, np.uint8)
+    onew = np.full((N, K // 32), 127, np.uint8)
+    assert np.array_equal(oracle.linear_f32acc(xq, one, wq, onew), oracle.linear(xq, one, wq, onew))

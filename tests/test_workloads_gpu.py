@@ -1,0 +1,67 @@
+"""The block workload at small widths (all rows compared): each linear of
+the block on its own, and the chained block output against the oracle's
+chain."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import assert_within_tol, bf16_bits, bf16_values, f16_bits
+from mxfp8_w8a8_quantized_b200 import synth
+from oracle_chain import OracleLinear, block_rows, chain_band
+
+pytestmark = pytest.mark.gpu
+
+HID, FFN, M, T = 512, 1024, 300, 64
+
+
+def _weights(seed, blk, hidden, ffn):
+    width = {synth.HIDDEN: hidden, synth.FFN: ffn}
+    out = {}
+    for i, (name, K, N, _) in enumerate(synth.block_linears()):
+        w = synth.weights_device(width[N], width[K], seed, 10 * blk + i, "cuda").cpu().numpy()
+        b = f16_bits(synth.bias_device(width[N], seed, 10 * blk + i, "cuda"))
+        out[name] = OracleLinear(w, b)
+    return out
+
+
+def test_small_block_linears_and_chain():
+    from mxfp8_w8a8_quantized_b200 import mxfp8
+    from mxfp8_w8a8_quantized_b200.workloads import Block, workspaces
+    seed = 7
+    x = synth.activations_device(M, HID, seed, 1000, "cuda")
+    ctx = synth.activations_device(T, HID, seed, 1001, "cuda")
+    blk = Block(seed, 0, "cuda", hidden=HID, ffn=FFN)
+    wa, wb = workspaces(M, T, "cuda", hidden=HID, ffn=FFN)
+    y, mid = blk.forward(x, ctx, wa, wb, keep=True)
+    torch.cuda.synchronize()
+    assert mxfp8.device_status() == 0
+    lin = _weights(seed, 0, HID, FFN)
+    xb = bf16_bits(x)
+    # linears fed from generator inputs: single-linear tolerance, all rows
+    for name, key in (("attn1.to_q", "q1"), ("attn1.to_k", "k1"), ("attn1.to_v", "v1")):
+        assert_within_tol(bf16_values(bf16_bits(mid[key])), lin[name].exact(xb), name)
+    cb = bf16_bits(ctx)
+    for name, key in (("attn2.to_k", "k2"), ("attn2.to_v", "v2")):
+        assert_within_tol(bf16_values(bf16_bits(mid[key])), lin[name].exact(cb), name)
+    # chained output: within the drift band of two admissible oracle chains
+    ok, stats = chain_band(bf16_values(bf16_bits(y)), bf16_values(block_rows(xb, lin)),
+                           bf16_values(block_rows(xb, lin, f32acc=True)))
+    assert ok, stats
+
+
+def test_workspace_reuse_does_not_leak_between_blocks():
+    """Two blocks in a row through the same workspaces equal the same two
+    blocks through fresh workspaces."""
+    from mxfp8_w8a8_quantized_b200.workloads import Block, workspaces
+    seed = 8
+    x = synth.activations_device(M, HID, seed, 1000, "cuda")
+    ctx = synth.activations_device(T, HID, seed, 1001, "cuda")
+    b0 = Block(seed, 0, "cuda", hidden=HID, ffn=FFN)
+    b1 = Block(seed, 1, "cuda", hidden=HID, ffn=FFN)
+    wa, wb = workspaces(M, T, "cuda", hidden=HID, ffn=FFN)
+    y_shared = b1.forward(b0.forward(x, ctx, wa, wb), ctx, wa, wb)
+    y_fresh = b1.forward(b0.forward(x, ctx, *workspaces(M, T, "cuda", hidden=HID, ffn=FFN)), ctx,
+                         *workspaces(M, T, "cuda", hidden=HID, ffn=FFN))
+    torch.cuda.synchronize()
+    assert torch.equal(y_shared, y_fresh)
