@@ -48,6 +48,9 @@ def parse(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOADS[0], choices=WORKLOADS)
+    ap.add_argument("--unfused", action="store_true",
+                    help="chained workloads: ffn.net.0.proj writes BF16 and GELU + quantization run as "
+                         "separate kernels (default: fused into its epilogue)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -239,29 +242,45 @@ class LinearWorkload:
         return torch.empty(self.mx.linear_workspace_bytes(self.M, self.K), dtype=torch.uint8, device=dev)
 
 
+def _gemm_bytes(M, K, N, quantized_out=False):
+    """Algorithmic HBM bytes of one GEMM launch: operands with their scales,
+    bias, and the output (BF16, or E4M3 codes + scales when the epilogue
+    quantizes for the next linear)."""
+    out = M * N * (1 + 1 / 32) if quantized_out else 2 * M * N
+    return M * K * (1 + 1 / 32) + N * K * (1 + 1 / 32) + out + 2 * N
+
+
+def _quant_bytes(M, K):
+    """Algorithmic HBM bytes of one activation quantization."""
+    return M * K * 3 + M * K // 32
+
+
 class FFNPairWorkload(LinearWorkload):
-    """ffn.net.0.proj -> GELU(tanh) -> ffn.net.2 at M tokens."""
+    """ffn.net.0.proj -> GELU(tanh) -> ffn.net.2 at M tokens.  Fused (the
+    default): ffn.net.0.proj's epilogue applies the GELU and quantizes for
+    ffn.net.2; otherwise GEMM, GELU kernel and quantizer run separately."""
 
     long_step = True
 
-    def __init__(self, name, M, seed, desc):
+    def __init__(self, name, M, seed, desc, fused=True):
         from mxfp8_w8a8_quantized_b200 import synth
         super().__init__(name, M, synth.HIDDEN, synth.FFN, seed, desc)
+        self.fused = fused
 
     def config(self):
-        return {"M": self.M, "hidden": self.K, "ffn": self.N}
+        return {"M": self.M, "hidden": self.K, "ffn": self.N,
+                "ffn0_epilogue": "gelu + quantize fused" if self.fused else "bf16 out; gelu, quantize separate"}
 
     def flops(self):
         return 2 * 2.0 * self.M * self.N * self.K
 
     def quant_bytes(self):
-        return self.M * (self.K + self.N) * 3 + self.M * (self.K + self.N) // 32
+        q = _quant_bytes(self.M, self.K)
+        return q if self.fused else q + _quant_bytes(self.M, self.N)
 
     def gemm_bytes(self):
         M, H, F = self.M, self.K, self.N
-        one = M * H * (1 + 1 / 32) + F * H * (1 + 1 / 32) + 2 * M * F + 2 * F
-        two = M * F * (1 + 1 / 32) + H * F * (1 + 1 / 32) + 2 * M * H + 2 * H
-        return one + two
+        return _gemm_bytes(M, H, F, quantized_out=self.fused) + _gemm_bytes(M, F, H)
 
     def setup(self, dev):
         from mxfp8_w8a8_quantized_b200 import mxfp8, synth
@@ -271,17 +290,21 @@ class FFNPairWorkload(LinearWorkload):
         self.x = synth.activations_device(M, H, s, 0, dev)
         self.l0 = QLinear.random(H, F, s, 1, dev)
         self.l2 = QLinear.random(F, H, s, 2, dev)
-        self.ws_ = Workspace(M * F, M, F, dev)
-        self.f = torch.empty((M, F), dtype=torch.bfloat16, device=dev)
+        self.wsx = Workspace(M * H, M, H, dev)
+        self.wsf = Workspace(M * F, M, F, dev)
+        self.f = None if self.fused else torch.empty((M, F), dtype=torch.bfloat16, device=dev)
         self.y = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
-        self.launches = 5
+        self.launches = 3 if self.fused else 5
 
     def _run(self, T, x, y):
         mx = self.mx
-        xq, xs = T("quant", self.ws_.quantize, x)
-        T("gemm", self.l0, xq, xs, out=self.f)
-        T("gelu", mx.gelu_tanh, self.f, out=self.f)
-        fq, fs = T("quant", self.ws_.quantize, self.f)
+        xq, xs = T("quant", self.wsx.quantize, x)
+        if self.fused:
+            fq, fs = T("gemm", self.l0.quantize_out, xq, xs, mx.ACT_GELU_TANH, self.wsf)
+        else:
+            T("gemm", self.l0, xq, xs, out=self.f)
+            T("gelu", mx.gelu_tanh, self.f, out=self.f)
+            fq, fs = T("quant", self.wsf.quantize, self.f)
         T("gemm", self.l2, fq, fs, out=y)
 
     def step(self, T):
@@ -295,28 +318,35 @@ class FFNPairWorkload(LinearWorkload):
 
 
 class BlocksWorkload(LinearWorkload):
-    """`nblocks` Wan blocks (10 quantized linears each) at M video / T text tokens."""
+    """`nblocks` Wan blocks (10 quantized linears each) at M video / T text
+    tokens; ffn.net.0.proj's epilogue fused with GELU + quantization unless
+    fused=False."""
 
     long_step = True
 
-    def __init__(self, name, M, T, nblocks, seed, desc):
+    def __init__(self, name, M, T, nblocks, seed, desc, fused=True):
         from mxfp8_w8a8_quantized_b200 import synth
         super().__init__(name, M, synth.HIDDEN, synth.FFN, seed, desc)
-        self.T, self.nblocks = T, nblocks
+        self.T, self.nblocks, self.fused = T, nblocks, fused
 
     def config(self):
-        return {"M": self.M, "text_tokens": self.T, "blocks": self.nblocks, "hidden": self.K, "ffn": self.N}
+        return {"M": self.M, "text_tokens": self.T, "blocks": self.nblocks, "hidden": self.K, "ffn": self.N,
+                "ffn0_epilogue": "gelu + quantize fused" if self.fused else "bf16 out; gelu, quantize separate"}
 
     def _per_block(self):
         from mxfp8_w8a8_quantized_b200 import synth
         fl, qb, gb = 0.0, 0.0, 0.0
-        for _, K, N, kind in synth.block_linears():
+        for name, K, N, kind in synth.block_linears():
             rows = self.M if kind == "video" else self.T
             fl += 2.0 * rows * K * N
-            gb += rows * K * (1 + 1 / 32) + N * K * (1 + 1 / 32) + 2 * rows * N + 2 * N
-        # distinct quantizations: x (q/k/v), v1, o1, ctx (k/v), q2, o2, gelu out
-        for rows, K in [(self.M, self.K)] * 5 + [(self.T, self.K), (self.M, self.N)]:
-            qb += rows * K * 3 + rows * K // 32
+            gb += _gemm_bytes(rows, K, N, quantized_out=self.fused and name == "ffn.net.0.proj")
+        # stand-alone quantizations: x (shared by q/k/v), v1, o1, ctx (shared
+        # by k/v), q2, o2, and the GELU output unless fused
+        quants = [(self.M, self.K)] * 5 + [(self.T, self.K)]
+        if not self.fused:
+            quants.append((self.M, self.N))
+        for rows, K in quants:
+            qb += _quant_bytes(rows, K)
         return fl, qb, gb
 
     def flops(self):
@@ -338,26 +368,13 @@ class BlocksWorkload(LinearWorkload):
         self.blocks = [Block(s, b, dev) for b in range(self.nblocks)]
         self.wa, self.wb = workspaces(self.M, self.T, dev)
         self.y = None
-        self.launches = self.nblocks * (10 + 7 + 1)
+        self.launches = self.nblocks * (16 if self.fused else 18)
 
     def _run(self, T, x):
-        from mxfp8_w8a8_quantized_b200.workloads import QLinear
-        orig = QLinear.__call__
-        wsq_a, wsq_b = self.wa.quantize, self.wb.quantize
-        try:
-            QLinear.__call__ = lambda lin, xq, xs, out=None: T("gemm", orig, lin, xq, xs, out=out)
-            self.wa.quantize = lambda t: T("quant", wsq_a, t)
-            self.wb.quantize = lambda t: T("quant", wsq_b, t)
-            gelu = self.mx.gelu_tanh
-            self.mx.gelu_tanh = lambda t, out=None: T("gelu", gelu, t, out=out)
-            y = x
-            for blk in self.blocks:
-                y = blk.forward(y, self.ctx, self.wa, self.wb)
-            return y
-        finally:
-            QLinear.__call__ = orig
-            self.wa.quantize, self.wb.quantize = wsq_a, wsq_b
-            self.mx.gelu_tanh = gelu
+        y = x
+        for blk in self.blocks:
+            y = blk.forward(y, self.ctx, self.wa, self.wb, fuse_ffn=self.fused, timer=T)
+        return y
 
     def step(self, T):
         self.y = self._run(T, self.x)
@@ -372,7 +389,7 @@ class BlocksWorkload(LinearWorkload):
         return None
 
 
-def make_workload(name):
+def make_workload(name, fused=True):
     from mxfp8_w8a8_quantized_b200 import synth
     H, F = synth.HIDDEN, synth.FFN
     M1, M2, T = synth.TOKENS_480P, synth.TOKENS_832x1104, synth.TEXT_TOKENS
@@ -385,18 +402,20 @@ def make_workload(name):
     if name == "ffn2_832x1104":
         return LinearWorkload(name, M2, F, H, 2, "Wan2.2 A14B ffn.net.2 at 832x1104, 81 frames")
     if name == "c2_ffn_pair_832x1104":
-        return FFNPairWorkload(name, M2, 2, "Wan2.2 A14B FFN pair (5120->13824->5120, GELU-tanh) at 832x1104")
+        return FFNPairWorkload(name, M2, 2, "Wan2.2 A14B FFN pair (5120->13824->5120, GELU-tanh) at 832x1104",
+                               fused=fused)
     if name == "c3_block_832x1104":
-        return BlocksWorkload(name, M2, T, 1, 3, "one Wan2.2 A14B block's 10 quantized linears at 832x1104")
+        return BlocksWorkload(name, M2, T, 1, 3, "one Wan2.2 A14B block's 10 quantized linears at 832x1104",
+                              fused=fused)
     if name == "c4_step_832x1104":
         return BlocksWorkload(name, M2, T, synth.BLOCKS, 4,
-                              "one denoising step: 40 blocks x 10 quantized linears at 832x1104")
+                              "one denoising step: 40 blocks x 10 quantized linears at 832x1104", fused=fused)
     raise ValueError(name)
 
 
 # ---------------------------------------------------------------- our arm
 def run_ours(args, ranks, dev):
-    wl = make_workload(args.workload)
+    wl = make_workload(args.workload, fused=not args.unfused)
     wl.setup(dev)
     stream = torch.cuda.current_stream(dev)
     mx = wl.mx

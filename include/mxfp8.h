@@ -65,6 +65,13 @@ typedef enum {
     MXFP8_SF_TCGEN05 = 1
 } mxfp8_sf_layout;
 
+/* Elementwise function applied to a layer's BF16 output before it is
+ * quantized for the next layer (mxfp8_gemm_quantize_out). */
+typedef enum {
+    MXFP8_ACT_NONE = 0,
+    MXFP8_ACT_GELU_TANH = 1   /* as mxfp8_gelu_tanh_bf16 */
+} mxfp8_activation;
+
 /* Human-readable name of a status.  Static storage; never NULL. */
 const char *mxfp8_status_str(mxfp8_status s);
 
@@ -141,10 +148,37 @@ mxfp8_status mxfp8_gemm_prequant(const void *Xq, const void *Xscale, int64_t M, 
  * GELU, tanh form, between ffn.net.0.proj and ffn.net.2 (the pages leave its
  * form open; this is the tanh approximation
  * 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))), evaluated in FP32 as
- * x / (1 + exp(-2u)), BF16 in and out, rounded to nearest even).
+ * x / (1 + exp(-2u)) with the hardware's approximate exp2 and reciprocal
+ * (relative error below 2^-16 before rounding), BF16 in and out, rounded to
+ * nearest even: within one BF16 ulp of the exact function).
  *   X, Y    BF16 [n] (Y may equal X), 16-byte aligned, n % 8 == 0.
  */
 mxfp8_status mxfp8_gelu_tanh_bf16(const void *X, void *Y, int64_t n, mxfp8_stream_t stream);
+
+/*
+ * The GEMM with the next linear's activation quantization in its epilogue
+ * (the optional fusion of the quantizer into the previous layer's epilogue,
+ * e.g. ffn.net.0.proj -> GELU -> ffn.net.2 of the model card's "Coverage per
+ * transformer").  The layer's BF16 output is not written; the result is
+ * bit-identical to
+ *     mxfp8_gemm_prequant(..., Y)
+ *     [mxfp8_gelu_tanh_bf16(Y, Y)]               when act == MXFP8_ACT_GELU_TANH
+ *     mxfp8_quantize(Y, M, N, N, Yq, Yscale, MXFP8_SF_TCGEN05)
+ * which it replaces, saving Y's BF16 write and the two passes over it.
+ *
+ *   Xq, Xscale, Wq, Wscale, bias   as mxfp8_gemm_prequant
+ *   act     MXFP8_ACT_NONE or MXFP8_ACT_GELU_TANH
+ *   Yq      E4M3 codes [M, N], row stride N (written), 16-byte aligned
+ *   Yscale  E8M0 scales of [M, N] in MXFP8_SF_TCGEN05 layout,
+ *           mxfp8_scale_bytes(M, N, MXFP8_SF_TCGEN05) bytes (written,
+ *           padding rows included), 16-byte aligned
+ * Requires K % 128 == 0 and N % 128 == 0 (the next linear's K), N > 0,
+ * M >= 0.  Errors as mxfp8_gemm_prequant; MXFP8_ERR_ARG for an unknown act.
+ */
+mxfp8_status mxfp8_gemm_quantize_out(const void *Xq, const void *Xscale, int64_t M, int64_t K,
+                                     const void *Wq, const void *Wscale, int64_t N,
+                                     const void *bias, int act, void *Yq, void *Yscale,
+                                     mxfp8_stream_t stream);
 
 /*
  * mxfp8_linear for callers that cannot allocate device memory.  The pages

@@ -17,7 +17,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmxfp8.so")
 
 SOURCES = ["mxfp8_quant.cu", "mxfp8_gemm.cu", "mxfp8_capi.cu", "mxfp8_noalloc.cu"]
-HEADERS = ["ptx.cuh"]
+HEADERS = ["ptx.cuh", "mx_element.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

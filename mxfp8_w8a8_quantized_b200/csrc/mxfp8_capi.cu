@@ -12,7 +12,8 @@ cudaError_t launch_quantize(const void *X, bool f32_in, int64_t M, int64_t K, in
                             bool sf_tc, cudaStream_t stream);
 cudaError_t launch_gelu(const void *X, void *Y, int64_t n, cudaStream_t stream);
 int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void *Wq, const void *Ws, int64_t N,
-                const void *bias, void *Y, cudaStream_t stream, unsigned long long timeout_ns, cudaError_t *err);
+                const void *bias, void *Y, int epi, void *S, cudaStream_t stream, unsigned long long timeout_ns,
+                cudaError_t *err);
 cudaError_t read_and_clear_status(unsigned int *out);
 } // namespace mx
 
@@ -142,10 +143,33 @@ mxfp8_status mxfp8_gemm_prequant(const void *Xq, const void *Xscale, int64_t M, 
     if (st != MXFP8_OK || M == 0)
         return st;
     cudaError_t e;
-    int r = mx::launch_gemm(Xq, Xscale, M, K, Wq, Wscale, N, bias, Y, reinterpret_cast<cudaStream_t>(stream),
-                            kWaitLimitNs, &e);
+    int r = mx::launch_gemm(Xq, Xscale, M, K, Wq, Wscale, N, bias, Y, 0, nullptr,
+                            reinterpret_cast<cudaStream_t>(stream), kWaitLimitNs, &e);
     if (r == 1)
         return MXFP8_ERR_CUDA; /* tensor map could not be encoded */
+    return r == 0 ? MXFP8_OK : from_cuda(e);
+}
+
+mxfp8_status mxfp8_gemm_quantize_out(const void *Xq, const void *Xscale, int64_t M, int64_t K, const void *Wq,
+                                     const void *Wscale, int64_t N, const void *bias, int act, void *Yq,
+                                     void *Yscale, mxfp8_stream_t stream)
+{
+    if (act != MXFP8_ACT_NONE && act != MXFP8_ACT_GELU_TANH)
+        return MXFP8_ERR_ARG;
+    mxfp8_status st = gemm_args(Xq, Xscale, M, K, Wq, Wscale, N, bias, Yq);
+    if (st != MXFP8_OK || M == 0)
+        return st;
+    if (!Yscale)
+        return MXFP8_ERR_ARG;
+    if (N % 128 != 0)
+        return MXFP8_ERR_SHAPE;
+    if (!aligned(Yscale, 16))
+        return MXFP8_ERR_ALIGN;
+    cudaError_t e;
+    int r = mx::launch_gemm(Xq, Xscale, M, K, Wq, Wscale, N, bias, Yq, act == MXFP8_ACT_GELU_TANH ? 2 : 1, Yscale,
+                            reinterpret_cast<cudaStream_t>(stream), kWaitLimitNs, &e);
+    if (r == 1)
+        return MXFP8_ERR_CUDA;
     return r == 0 ? MXFP8_OK : from_cuda(e);
 }
 

@@ -60,6 +60,7 @@
 #include <cstdint>
 #include <cstdlib>
 
+#include "mx_element.cuh"
 #include "ptx.cuh"
 
 namespace mx {
@@ -86,6 +87,13 @@ constexpr uint32_t SUSPEND_PIPE = MX_SUSPEND_PIPE;
 constexpr uint32_t SUSPEND_EPI = MX_SUSPEND_EPI;
 constexpr int PREFETCH_KB = MX_PREFETCH_KB; /* K steps the L2 prefetch runs ahead of the loads (0 = off) */
 constexpr uint32_t ST_TIMEOUT = 1u;
+
+/* What the epilogue writes. */
+enum EpiMode : int {
+    EPI_BF16 = 0,       /* Y = BF16(acc + bias) */
+    EPI_QUANT = 1,      /* MXFP8 codes + scales of BF16(acc + bias) for the next linear */
+    EPI_QUANT_GELU = 2, /* MXFP8 codes + scales of BF16(GELU(BF16(acc + bias))) */
+};
 
 template <bool PAIR>
 struct Cfg {
@@ -123,8 +131,11 @@ __device__ unsigned int g_mx_status = 0;
 
 struct GemmParams {
     const __half *bias;   /* [N] or null */
-    __nv_bfloat16 *Y;     /* [M, N] */
+    __nv_bfloat16 *Y;     /* [M, N] (EPI_BF16) */
+    uint8_t *S;           /* output scales, tensor-core layout of [M, N] (quantizing modes) */
     int M, N, K;
+    int m_pad;            /* M rounded up to 128: rows that own scale bytes */
+    int sf_kgroups;       /* N / 128: scale atoms per 128 output rows */
     int num_m, num_n;     /* output tiles */
     unsigned long long timeout_ns;
 };
@@ -164,7 +175,163 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, unsi
     }
 }
 
-template <bool PAIR>
+/* Epilogue writing Y = BF16(acc + bias): bias + BF16 rounding, 32 columns at
+ * a time, staged through a 64-byte-swizzled smem box and written by one TMA
+ * store per warp -- scattered per-row global stores would occupy the L1 /
+ * shared-memory data path that feeds the tensor core. */
+__device__ __forceinline__ void epilogue_bf16(const uint32_t (&acc)[128], const GemmParams &p,
+                                              const CUtensorMap *tmap_y, int row0, int col0, int lane,
+                                              uint32_t buf, uint32_t rowbase, uint32_t swz)
+{
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const int colc = col0 + 32 * c;
+        if (row0 >= p.M || colc >= p.N) /* whole box outside Y: nothing to store */
+            continue;
+        if (lane == 0)
+            bulk_wait_group_read0(); /* previous box has left the buffer */
+        __syncwarp();
+#pragma unroll
+        for (int j8 = 0; j8 < 4; ++j8) {
+            const int col = colc + 8 * j8;
+            float b[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (p.bias && col < p.N) {
+                const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(p.bias + col));
+                const __half2 *bh = reinterpret_cast<const __half2 *>(&bv);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 f2 = __half22float2(bh[j]);
+                    b[2 * j] = f2.x;
+                    b[2 * j + 1] = f2.y;
+                }
+            }
+            uint32_t o[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int a = 32 * c + 8 * j8 + 2 * j;
+                __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(acc[a]) + b[2 * j],
+                                                         __uint_as_float(acc[a + 1]) + b[2 * j + 1]);
+                o[j] = *reinterpret_cast<uint32_t *>(&v);
+            }
+            st_shared_v4(rowbase + ((((uint32_t)j8) ^ swz) << 4), o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmap_y, colc, row0, buf);
+            bulk_commit_group();
+        }
+    }
+}
+
+/*
+ * Epilogue that quantizes the layer's output for the next linear instead of
+ * writing it: per row, BF16(acc + bias) (then BF16(GELU(.)) when GELU is
+ * set) is exactly what the stand-alone path writes to Y, and the MX
+ * quantization of those BF16 values is exactly what the stand-alone
+ * quantizer computes from Y.  A thread owns one output row of the warp's
+ * 128 columns, i.e. four whole 32-element blocks, so the block maximum is a
+ * per-thread reduction.  The accumulator is packed to BF16 pairs first,
+ * which halves the registers it holds and leaves room for the GELU's
+ * independent chains.  Codes leave as two 32-row x 64-byte boxes through the
+ * warp's swizzled staging buffer (TMA store, clipped at M); the four scale
+ * bytes of the row form one 32-bit word of the tensor-core scale layout
+ * (row r of atom (r / 128, col / 128) at byte (r % 32) * 16 + (r / 32 % 4) *
+ * 4), written directly.  Rows in [M, m_pad) get zero scale words, as the
+ * stand-alone quantizer writes for its padding rows.
+ */
+template <bool GELU>
+__device__ __forceinline__ void epilogue_quantize(const uint32_t (&acc)[128], const GemmParams &p,
+                                                  const CUtensorMap *tmap_q, int row0, int col0, int lane,
+                                                  uint32_t buf, uint32_t rowbase, uint32_t swz)
+{
+    if (col0 >= p.N || row0 >= p.m_pad) /* warp-uniform: N % 128 == 0 */
+        return;
+    const int row = row0 + lane;
+    uint32_t sword = 0u;
+    if (row0 < p.M) {
+        uint32_t y[64]; /* BF16 pairs: columns 2i, 2i + 1 */
+#pragma unroll
+        for (int j8 = 0; j8 < 16; ++j8) {
+            float b[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (p.bias) {
+                const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(p.bias + col0 + 8 * j8));
+                const __half2 *bh = reinterpret_cast<const __half2 *>(&bv);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 f2 = __half22float2(bh[j]);
+                    b[2 * j] = f2.x;
+                    b[2 * j + 1] = f2.y;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int a = 8 * j8 + 2 * j;
+                y[4 * j8 + j] = f32x2_to_bf16x2(f2_add(f2_pack(__uint_as_float(acc[a]), __uint_as_float(acc[a + 1])),
+                                                       f2_pack(b[2 * j], b[2 * j + 1])));
+            }
+        }
+        /* one 32-column block per iteration, always from y[0 .. 15]; the
+         * remaining words move down after each block */
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int g = c & 1; /* position inside the 64-column code box */
+            if (g == 0) {
+                if (lane == 0)
+                    bulk_wait_group_read0(); /* previous box has left the buffer */
+                __syncwarp();
+            }
+            if constexpr (GELU) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    y[i] = gelu_tanh_bf16x2(y[i]);
+            }
+            /* non-negative BF16 bit patterns order like their values */
+            uint32_t m2 = 0u;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                m2 = __vmaxu2(m2, y[i] & 0x7FFF7FFFu);
+            const uint32_t sb = scale_byte_from_amax(max(m2 << 16, m2 & 0xFFFF0000u));
+            sword |= sb << (8 * c);
+            uint32_t o[8];
+            if (sb == 0xFFu) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    o[i] = 0x7F7F7F7Fu;
+            } else {
+                const float m = inv_scale(sb);
+                const f32x2 mm = f2_pack(m, m);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float c0, c1, c2, c3;
+                    f2_unpack(f2_mul(bf16x2_to_f32x2(y[2 * i]), mm), c0, c1);
+                    f2_unpack(f2_mul(bf16x2_to_f32x2(y[2 * i + 1]), mm), c2, c3);
+                    o[i] = pack4_e4m3(c0, c1, c2, c3);
+                }
+            }
+            st_shared_v4(rowbase + ((((uint32_t)(2 * g)) ^ swz) << 4), o[0], o[1], o[2], o[3]);
+            st_shared_v4(rowbase + ((((uint32_t)(2 * g + 1)) ^ swz) << 4), o[4], o[5], o[6], o[7]);
+            if (g == 1) {
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(tmap_q, col0 + 64 * (c >> 1), row0, buf);
+                    bulk_commit_group();
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 48; ++i)
+                y[i] = y[i + 16];
+        }
+    }
+    if (row < p.m_pad) {
+        const int64_t off = (((int64_t)(row >> 7) * p.sf_kgroups + (col0 >> 7)) << 9) + ((row & 31) << 4) +
+                            (((row >> 5) & 3) << 2);
+        *reinterpret_cast<uint32_t *>(p.S + off) = row < p.M ? sword : 0u;
+    }
+}
+
+template <bool PAIR, int EPI>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
@@ -412,54 +579,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     mbar_arrive(bar_tempty);
             }
 
-            /* bias + BF16 rounding, 32 columns at a time, staged through a
-             * 64-byte-swizzled smem box and written by one TMA store per
-             * warp: scattered per-row global stores would occupy the L1 /
-             * shared-memory data path that feeds the tensor core. */
             const int row0 = mb * C::TILE_M + (int)(rank * 128u) + 32 * q;
             const int col0 = nb * C::TILE_N + h * 128;
             const uint32_t buf = sbase + C::OFF_EPI + (uint32_t)(warp - 2) * C::EPI_BUF;
             const uint32_t rowbase = buf + (uint32_t)lane * 64u;
             const uint32_t swz = ((uint32_t)lane >> 1) & 3u;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int colc = col0 + 32 * c;
-                if (row0 >= p.M || colc >= p.N) /* whole box outside Y: nothing to store */
-                    continue;
-                if (lane == 0)
-                    bulk_wait_group_read0(); /* previous box has left the buffer */
-                __syncwarp();
-#pragma unroll
-                for (int j8 = 0; j8 < 4; ++j8) {
-                    const int col = colc + 8 * j8;
-                    float b[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                    if (p.bias && col < p.N) {
-                        const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(p.bias + col));
-                        const __half2 *bh = reinterpret_cast<const __half2 *>(&bv);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float2 f2 = __half22float2(bh[j]);
-                            b[2 * j] = f2.x;
-                            b[2 * j + 1] = f2.y;
-                        }
-                    }
-                    uint32_t o[4];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int a = 32 * c + 8 * j8 + 2 * j;
-                        __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(acc[a]) + b[2 * j],
-                                                                 __uint_as_float(acc[a + 1]) + b[2 * j + 1]);
-                        o[j] = *reinterpret_cast<uint32_t *>(&v);
-                    }
-                    st_shared_v4(rowbase + ((((uint32_t)j8) ^ swz) << 4), o[0], o[1], o[2], o[3]);
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&tmap_y, colc, row0, buf);
-                    bulk_commit_group();
-                }
-            }
+            if constexpr (EPI == EPI_BF16)
+                epilogue_bf16(acc, p, &tmap_y, row0, col0, lane, buf, rowbase, swz);
+            else
+                epilogue_quantize<EPI == EPI_QUANT_GELU>(acc, p, &tmap_y, row0, col0, lane, buf, rowbase, swz);
         }
         if (lane == 0)
             bulk_wait_group0(); /* stores complete before the CTA exits */
@@ -547,11 +675,28 @@ static bool make_output_map(CUtensorMap *m, void *base, int64_t M, int64_t N)
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+/* MXFP8 codes out [M, N] (quantizing epilogues): box 64 bytes x 32 rows,
+ * 64-byte swizzle (same staging layout as the BF16 boxes); clipped at M. */
+static bool make_codes_out_map(CUtensorMap *m, void *base, int64_t M, int64_t N)
+{
+    PFN_encodeTiled enc = get_encode_fn();
+    if (!enc)
+        return false;
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)N};
+    cuuint32_t box[2] = {64, 32};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct DevInfo {
     bool init = false;
     int sms = 148;
-    int max_pair_clusters = 0; /* 0: pairs unavailable */
-    bool attr_single = false, attr_pair = false;
+    bool pair_checked = false;
+    int max_pair_clusters = 0;   /* 0: pairs unavailable */
+    bool attr[2][3] = {};        /* [PAIR][EPI]: shared-memory attribute set */
 };
 static DevInfo g_dev[64];
 
@@ -570,26 +715,88 @@ static DevInfo *dev_info()
     return &d;
 }
 
-template <bool PAIR>
-static cudaError_t launch_variant(const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorMap &msa,
+template <bool PAIR, int EPI>
+static cudaError_t ensure_attr(DevInfo *d)
+{
+    if (d->attr[PAIR][EPI])
+        return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(mxfp8_gemm_kernel<PAIR, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Cfg<PAIR>::SMEM_BYTES);
+    if (e == cudaSuccess)
+        d->attr[PAIR][EPI] = true;
+    return e;
+}
+
+static void pair_config(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attr, unsigned grid, cudaStream_t stream)
+{
+    cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(GEMM_THREADS);
+    cfg.dynamicSmemBytes = Cfg<true>::SMEM_BYTES;
+    cfg.stream = stream;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+}
+
+/* How many CTA pairs can be resident at once (0: pairs unavailable). */
+static void check_pairs(DevInfo *d)
+{
+    if (d->pair_checked)
+        return;
+    d->pair_checked = true;
+    if (ensure_attr<true, EPI_BF16>(d) != cudaSuccess) {
+        cudaGetLastError();
+        return;
+    }
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attr[1];
+    pair_config(cfg, attr, 2 * (unsigned)d->sms, nullptr);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, mxfp8_gemm_kernel<true, EPI_BF16>, &cfg) == cudaSuccess)
+        d->max_pair_clusters = n;
+    else
+        cudaGetLastError(); /* clear; fall back to single CTAs */
+}
+
+template <bool PAIR, int EPI>
+static cudaError_t launch_variant(DevInfo *d, const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorMap &msa,
                                   const CUtensorMap &msb, const CUtensorMap &my, const GemmParams &p, int grid,
                                   cudaStream_t stream)
 {
-    cudaLaunchConfig_t cfg = {};
+    cudaError_t e = ensure_attr<PAIR, EPI>(d);
+    if (e != cudaSuccess)
+        return e;
+    cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attr[1];
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(GEMM_THREADS);
-    cfg.dynamicSmemBytes = Cfg<PAIR>::SMEM_BYTES;
-    cfg.stream = stream;
     if (PAIR) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        pair_config(cfg, attr, (unsigned)grid, stream);
+    } else {
+        cfg = {};
+        cfg.gridDim = dim3((unsigned)grid);
+        cfg.blockDim = dim3(GEMM_THREADS);
+        cfg.dynamicSmemBytes = Cfg<PAIR>::SMEM_BYTES;
+        cfg.stream = stream;
     }
-    return cudaLaunchKernelEx(&cfg, mxfp8_gemm_kernel<PAIR>, ma, mb, msa, msb, my, p);
+    return cudaLaunchKernelEx(&cfg, mxfp8_gemm_kernel<PAIR, EPI>, ma, mb, msa, msb, my, p);
+}
+
+template <bool PAIR>
+static cudaError_t launch_mode(DevInfo *d, int epi, const CUtensorMap &ma, const CUtensorMap &mb,
+                               const CUtensorMap &msa, const CUtensorMap &msb, const CUtensorMap &my,
+                               const GemmParams &p, int grid, cudaStream_t stream)
+{
+    switch (epi) {
+    case EPI_QUANT:
+        return launch_variant<PAIR, EPI_QUANT>(d, ma, mb, msa, msb, my, p, grid, stream);
+    case EPI_QUANT_GELU:
+        return launch_variant<PAIR, EPI_QUANT_GELU>(d, ma, mb, msa, msb, my, p, grid, stream);
+    default:
+        return launch_variant<PAIR, EPI_BF16>(d, ma, mb, msa, msb, my, p, grid, stream);
+    }
 }
 
 /* Whether the CTA-pair variant is used: on unless MXFP8_GEMM_PAIR=0. */
@@ -603,9 +810,15 @@ static bool pair_enabled()
     return v == 1;
 }
 
-/* 0 ok, 1 tensor-map failure, 2 CUDA error (in *err). */
+/*
+ * epi = 0: Y is BF16 [M, N], S unused.  epi = 1 / 2: Y receives E4M3 codes
+ * [M, N] and S the tensor-core scales of [M, N] (2: GELU before the
+ * quantization); N % 128 == 0.
+ * Returns 0 ok, 1 tensor-map failure, 2 CUDA error (in *err).
+ */
 int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void *Wq, const void *Ws, int64_t N,
-                const void *bias, void *Y, cudaStream_t stream, unsigned long long timeout_ns, cudaError_t *err)
+                const void *bias, void *Y, int epi, void *S, cudaStream_t stream, unsigned long long timeout_ns,
+                cudaError_t *err)
 {
     *err = cudaSuccess;
     if (M == 0)
@@ -615,71 +828,44 @@ int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void
         *err = cudaErrorInvalidDevice;
         return 2;
     }
-    cudaError_t e;
     bool pair = pair_enabled();
-    if (pair && !d->attr_pair) {
-        e = cudaFuncSetAttribute(mxfp8_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)Cfg<true>::SMEM_BYTES);
-        if (e == cudaSuccess) {
-            cudaLaunchConfig_t cfg = {};
-            cudaLaunchAttribute attr[1];
-            cfg.gridDim = dim3(2 * (unsigned)d->sms);
-            cfg.blockDim = dim3(GEMM_THREADS);
-            cfg.dynamicSmemBytes = Cfg<true>::SMEM_BYTES;
-            attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = 2;
-            attr[0].val.clusterDim.y = 1;
-            attr[0].val.clusterDim.z = 1;
-            cfg.attrs = attr;
-            cfg.numAttrs = 1;
-            int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, mxfp8_gemm_kernel<true>, &cfg) == cudaSuccess)
-                d->max_pair_clusters = n;
-            else
-                cudaGetLastError(); /* clear; fall back to single CTAs */
-        } else {
-            cudaGetLastError();
-        }
-        d->attr_pair = true;
-    }
-    if (pair && d->max_pair_clusters <= 0)
-        pair = false;
-    if (!pair && !d->attr_single) {
-        e = cudaFuncSetAttribute(mxfp8_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)Cfg<false>::SMEM_BYTES);
-        if (e != cudaSuccess) {
-            *err = e;
-            return 2;
-        }
-        d->attr_single = true;
+    if (pair) {
+        check_pairs(d);
+        if (d->max_pair_clusters <= 0)
+            pair = false;
     }
 
     const uint32_t b_rows = pair ? Cfg<true>::B_ROWS : Cfg<false>::B_ROWS;
     CUtensorMap ma, mb, msa, msb, my;
+    const bool out_ok = epi == EPI_BF16 ? make_output_map(&my, Y, M, N) : make_codes_out_map(&my, Y, M, N);
     if (!make_operand_map(&ma, Xq, M, K, 128) || !make_operand_map(&mb, Wq, N, K, b_rows) ||
-        !make_scale_map(&msa, Xs, M, K, 1) || !make_scale_map(&msb, Ws, N, K, 2) || !make_output_map(&my, Y, M, N))
+        !make_scale_map(&msa, Xs, M, K, 1) || !make_scale_map(&msb, Ws, N, K, 2) || !out_ok)
         return 1;
     GemmParams p;
     p.bias = static_cast<const __half *>(bias);
     p.Y = static_cast<__nv_bfloat16 *>(Y);
+    p.S = static_cast<uint8_t *>(S);
     p.M = (int)M;
     p.N = (int)N;
     p.K = (int)K;
+    p.m_pad = (int)((M + 127) / 128 * 128);
+    p.sf_kgroups = (int)(N / 128);
     const int tile_m = pair ? Cfg<true>::TILE_M : Cfg<false>::TILE_M;
     p.num_m = (int)((M + tile_m - 1) / tile_m);
     p.num_n = (int)((N + 255) / 256);
     p.timeout_ns = timeout_ns;
     const int tiles = p.num_m * p.num_n;
+    cudaError_t e;
     if (pair) {
         int clusters = d->max_pair_clusters;
         if (clusters > tiles)
             clusters = tiles;
-        e = launch_variant<true>(ma, mb, msa, msb, my, p, 2 * clusters, stream);
+        e = launch_mode<true>(d, epi, ma, mb, msa, msb, my, p, 2 * clusters, stream);
     } else {
         int grid = d->sms;
         if (grid > tiles)
             grid = tiles;
-        e = launch_variant<false>(ma, mb, msa, msb, my, p, grid, stream);
+        e = launch_mode<false>(d, epi, ma, mb, msa, msb, my, p, grid, stream);
     }
     if (e != cudaSuccess) {
         *err = e;

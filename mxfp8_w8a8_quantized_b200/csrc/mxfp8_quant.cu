@@ -29,6 +29,8 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "mx_element.cuh"
+
 namespace mx {
 
 #ifndef MX_QUNROLL
@@ -39,28 +41,6 @@ namespace mx {
 #endif
 constexpr int QTHREADS = 256;
 constexpr int QUNROLL = MX_QUNROLL;     /* row segments in flight per warp */
-
-/* Scale byte from the bit pattern of amax as a binary32 (sign cleared). */
-__device__ __forceinline__ uint32_t scale_byte_from_amax(uint32_t abits)
-{
-    uint32_t ef = abits >> 23;
-    if (ef >= 255u)
-        return 0xFFu;                 /* Inf / NaN in the block */
-    return ef > 8u ? ef - 8u : 0u;    /* e = (ef - 127) - 8, clamped at -127 */
-}
-
-/* 2^-e as a binary32 for a finite scale byte b (e = b - 127, b <= 246). */
-__device__ __forceinline__ float inv_scale(uint32_t b)
-{
-    return __uint_as_float((254u - b) << 23);
-}
-
-__device__ __forceinline__ uint32_t pack4_e4m3(float a, float b, float c, float d)
-{
-    __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
-    __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
-    return (uint32_t)lo | ((uint32_t)hi << 16);
-}
 
 /* 16 consecutive elements of one row: one lane's share of a row segment. */
 template <bool F32_IN>
@@ -218,29 +198,13 @@ __global__ void __launch_bounds__(QTHREADS, MX_QMINBLOCKS) mx_quantize_kernel(co
 }
 
 /* ------------------------------------------------------------------ GELU */
-__device__ __forceinline__ float gelu_tanh_f32(float x)
-{
-    /* 0.5 x (1 + tanh(u)) == x sigmoid(2u),  u = sqrt(2/pi)(x + 0.044715 x^3);
-     * the exponential is taken of -|2u| so that it never overflows: for very
-     * negative x the result underflows gradually instead of becoming -0. */
-    const float u = 0.7978845608028654f * (x + 0.044715f * x * x * x);
-    const float t = expf(-fabsf(2.0f * u));
-    return u >= 0.0f ? x / (1.0f + t) : x * t / (1.0f + t);
-}
-
 __global__ void __launch_bounds__(256) gelu_tanh_bf16_kernel(const uint4 *__restrict__ X, uint4 *__restrict__ Y,
                                                              int64_t n8)
 {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
-        uint4 v = X[i];
-        uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            float lo = gelu_tanh_f32(__uint_as_float(w[j] << 16));
-            float hi = gelu_tanh_f32(__uint_as_float(w[j] & 0xFFFF0000u));
-            __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
-            w[j] = *reinterpret_cast<uint32_t *>(&p);
-        }
+        const uint4 v = X[i];
+        const uint32_t w[4] = {gelu_tanh_bf16x2(v.x), gelu_tanh_bf16x2(v.y), gelu_tanh_bf16x2(v.z),
+                               gelu_tanh_bf16x2(v.w)};
         Y[i] = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }

@@ -42,15 +42,20 @@ _lib.mxfp8_gelu_tanh_bf16.argtypes = [_P, _P, _I64, _P]
 _lib.mxfp8_gelu_tanh_bf16.restype = ctypes.c_int
 _lib.mxfp8_linear_noalloc.argtypes = [_P, _I64, _I64, _P, _P, _I64, _P, _P, _P]
 _lib.mxfp8_linear_noalloc.restype = ctypes.c_int
+_lib.mxfp8_gemm_quantize_out.argtypes = [_P, _P, _I64, _I64, _P, _P, _I64, _P, ctypes.c_int, _P, _P, _P]
+_lib.mxfp8_gemm_quantize_out.restype = ctypes.c_int
 _lib.mxfp8_device_status.argtypes = [_P]
 _lib.mxfp8_device_status.restype = ctypes.c_int
 
 SF_ROWMAJOR = 0
 SF_TCGEN05 = 1
+ACT_NONE = 0
+ACT_GELU_TANH = 1
 
 EXPORTS = ("mxfp8_status_str", "mxfp8_scale_bytes", "mxfp8_quantize", "mxfp8_quantize_weight_f32",
            "mxfp8_linear_workspace_bytes", "mxfp8_linear", "mxfp8_gemm_prequant",
-           "mxfp8_gelu_tanh_bf16", "mxfp8_device_status", "mxfp8_linear_noalloc")
+           "mxfp8_gelu_tanh_bf16", "mxfp8_device_status", "mxfp8_linear_noalloc",
+           "mxfp8_gemm_quantize_out")
 
 
 class MXFP8Error(RuntimeError):
@@ -155,6 +160,21 @@ def gemm_prequant(xq, xscale, wq, wscale, bias=None, out=None):
     _check(_lib.mxfp8_gemm_prequant(_ptr(xq), _ptr(xscale), M, K, _ptr(wq), _ptr(wscale), N,
                                     _ptr(bias), _ptr(out), _stream()), "mxfp8_gemm_prequant")
     return out
+
+
+def gemm_quantize_out(xq, xscale, wq, wscale, bias=None, act=ACT_NONE, codes=None, scales=None):
+    """The next linear's quantized input straight from this linear's GEMM:
+    (E4M3 codes uint8 [M, N], tensor-core scales) of BF16(act(BF16(acc + bias)))
+    without writing the BF16 output (act: ACT_NONE or ACT_GELU_TANH)."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    if codes is None:
+        codes = torch.empty((M, N), dtype=torch.uint8, device=xq.device)
+    if scales is None:
+        scales = torch.empty(max(scale_bytes(M, N), 1), dtype=torch.uint8, device=xq.device)
+    _check(_lib.mxfp8_gemm_quantize_out(_ptr(xq), _ptr(xscale), M, K, _ptr(wq), _ptr(wscale), N, _ptr(bias),
+                                        act, _ptr(codes), _ptr(scales), _stream()), "mxfp8_gemm_quantize_out")
+    return codes, scales
 
 
 def gelu_tanh(x: torch.Tensor, out=None):

@@ -18,6 +18,13 @@ replaced by stand-ins that keep every shape):
     y  = ffn.net.2(g)                   [M, 5120]  -> next block's x
 
 Every linear quantizes its BF16 input dynamically (MXFP8) before the GEMM.
+With fuse_ffn (the default), ffn.net.0.proj's epilogue applies the GELU and
+quantizes for ffn.net.2 itself (mxfp8_gemm_quantize_out): f and g are never
+written, and the result is bit-identical to the separate kernels.
+
+Every kernel call goes through `timer(kind, fn, *args)` ("quant", "gemm" or
+"gelu"), which the benchmark uses to time each kind; by default it just
+calls fn.
 """
 import torch
 
@@ -43,6 +50,12 @@ class QLinear:
     def __call__(self, xq, xs, out=None):
         return mxfp8.gemm_prequant(xq, xs, self.wq, self.ws, self.bias, out=out)
 
+    def quantize_out(self, xq, xs, act, dest):
+        """The next linear's MXFP8 input (codes, scales) from this GEMM's
+        epilogue, into Workspace `dest`."""
+        codes, scales = dest.views(xq.shape[0], self.N)
+        return mxfp8.gemm_quantize_out(xq, xs, self.wq, self.ws, self.bias, act=act, codes=codes, scales=scales)
+
 
 class Workspace:
     """Reusable activation-quantization buffers (codes + scales)."""
@@ -51,10 +64,12 @@ class Workspace:
         self.codes = torch.empty(max_elems, dtype=torch.uint8, device=device)
         self.scales = torch.empty(mxfp8.scale_bytes(max_rows, K_max), dtype=torch.uint8, device=device)
 
+    def views(self, M, K):
+        """(codes [M, K], tensor-core scales) views of the buffers."""
+        return self.codes[: M * K].view(M, K), self.scales[: mxfp8.scale_bytes(M, K)]
+
     def quantize(self, x):
-        M, K = x.shape
-        codes = self.codes[: M * K].view(M, K)
-        scales = self.scales[: mxfp8.scale_bytes(M, K)]
+        codes, scales = self.views(*x.shape)
         return mxfp8.quantize(x, codes=codes, scales=scales)
 
 
@@ -68,27 +83,38 @@ class Block:
         for i, (name, K, N, _) in enumerate(synth.block_linears()):
             self.lin[name] = QLinear.random(width[K], width[N], seed, 10 * block_index + i, device)
 
-    def forward(self, x, ctx, ws_a, ws_b, keep=False):
+    def forward(self, x, ctx, ws_a, ws_b, keep=False, fuse_ffn=True, timer=None):
         """x [M, hidden], ctx [T, hidden] BF16.  ws_a / ws_b: two Workspaces
         (two live quantized activations at most).  Returns y, plus every
-        intermediate when keep=True."""
+        intermediate when keep=True (g only without fuse_ffn)."""
         L = self.lin
-        xq, xs = ws_a.quantize(x)
-        q1 = L["attn1.to_q"](xq, xs)
-        k1 = L["attn1.to_k"](xq, xs)
-        v1 = L["attn1.to_v"](xq, xs)
-        o1 = L["attn1.to_out"](*ws_b.quantize(v1))
-        q2 = L["attn2.to_q"](*ws_a.quantize(o1))
-        cq, cs = ws_b.quantize(ctx)
-        k2 = L["attn2.to_k"](cq, cs)
-        v2 = L["attn2.to_v"](cq, cs)
-        o2 = L["attn2.to_out"](*ws_a.quantize(q2))
-        f = L["ffn.net.0.proj"](*ws_b.quantize(o2))
-        mxfp8.gelu_tanh(f, out=f)
-        y = L["ffn.net.2"](*ws_a.quantize(f))
+        T = timer or _call
+        xq, xs = T("quant", ws_a.quantize, x)
+        q1 = T("gemm", L["attn1.to_q"], xq, xs)
+        k1 = T("gemm", L["attn1.to_k"], xq, xs)
+        v1 = T("gemm", L["attn1.to_v"], xq, xs)
+        o1 = T("gemm", L["attn1.to_out"], *T("quant", ws_b.quantize, v1))
+        q2 = T("gemm", L["attn2.to_q"], *T("quant", ws_a.quantize, o1))
+        cq, cs = T("quant", ws_b.quantize, ctx)
+        k2 = T("gemm", L["attn2.to_k"], cq, cs)
+        v2 = T("gemm", L["attn2.to_v"], cq, cs)
+        o2 = T("gemm", L["attn2.to_out"], *T("quant", ws_a.quantize, q2))
+        oq, os_ = T("quant", ws_b.quantize, o2)
+        g = None
+        if fuse_ffn:
+            gq, gs = T("gemm", L["ffn.net.0.proj"].quantize_out, oq, os_, mxfp8.ACT_GELU_TANH, ws_a)
+        else:
+            g = T("gemm", L["ffn.net.0.proj"], oq, os_)
+            T("gelu", mxfp8.gelu_tanh, g, out=g)
+            gq, gs = T("quant", ws_a.quantize, g)
+        y = T("gemm", L["ffn.net.2"], gq, gs)
         if keep:
-            return y, dict(q1=q1, k1=k1, v1=v1, o1=o1, q2=q2, k2=k2, v2=v2, o2=o2, g=f)
+            return y, dict(q1=q1, k1=k1, v1=v1, o1=o1, q2=q2, k2=k2, v2=v2, o2=o2, g=g)
         return y
+
+
+def _call(kind, fn, *args, **kw):
+    return fn(*args, **kw)
 
 
 def workspaces(M, T, device, hidden=synth.HIDDEN, ffn=synth.FFN):

@@ -84,3 +84,20 @@ def test_workload_accounting():
     expect = 2.0 * (6 * 75348 * 5120 * 5120 + 2 * 512 * 5120 * 5120 + 2 * 75348 * 5120 * 13824)
     assert blk.flops() == pytest.approx(expect)
     assert step.flops() == pytest.approx(40 * expect)
+
+
+def test_fused_accounting():
+    """The fused FFN epilogue removes one quantization per block and writes
+    E4M3 codes + scales instead of BF16 for ffn.net.0.proj."""
+    sys.path.insert(0, ROOT)
+    import bench
+    M, H, F = 75348, 5120, 13824
+    fused = bench.make_workload("c2_ffn_pair_832x1104")
+    plain = bench.make_workload("c2_ffn_pair_832x1104", fused=False)
+    assert fused.flops() == plain.flops()
+    assert plain.quant_bytes() - fused.quant_bytes() == M * F * 3 + M * F // 32
+    assert plain.gemm_bytes() - fused.gemm_bytes() == pytest.approx(M * F * (2 - (1 + 1 / 32)))
+    bf = bench.make_workload("c3_block_832x1104")
+    bp = bench.make_workload("c3_block_832x1104", fused=False)
+    assert bp.quant_bytes() - bf.quant_bytes() == M * F * 3 + M * F // 32
+    assert bf.flops() == bp.flops()

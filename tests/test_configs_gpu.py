@@ -156,6 +156,29 @@ def test_ffn_pair_832x1104_full_size(mx):
     check_chain("ffn_pair_chain", got, ref64, ref32)
 
 
+def test_ffn0_fused_epilogue_832x1104_full_size(mx):
+    """ffn.net.0.proj at M = 75348 with GELU + quantization in its epilogue:
+    all 1.04 G codes and all scale bytes equal GEMM -> GELU -> quantize."""
+    M, H, F, seed = synth.TOKENS_832x1104, synth.HIDDEN, synth.FFN, 5
+    x = synth.activations_device(M, H, seed, 0, DEV)
+    w = synth.weights_device(F, H, seed, 1, DEV)
+    b = synth.bias_device(F, seed, 1, DEV)
+    wq, ws = mx.quantize_weight(w)
+    del w
+    xq, xs = mx.quantize(x)
+    del x
+    cf, sf = mx.gemm_quantize_out(xq, xs, wq, ws, b, act=mx.ACT_GELU_TANH)
+    y = mx.gemm_prequant(xq, xs, wq, ws, b)
+    mx.gelu_tanh(y, out=y)
+    cs, ss = mx.quantize(y)
+    torch.cuda.synchronize()
+    assert mx.device_status() == 0
+    assert torch.equal(cf, cs)
+    assert torch.equal(sf, ss)
+    del y, cf, cs
+    torch.cuda.empty_cache()
+
+
 def test_block_832x1104_full_size(mx):
     """One block's ten linears at M = 75348 video / 512 text tokens."""
     from mxfp8_w8a8_quantized_b200.workloads import Block, workspaces

@@ -65,3 +65,17 @@ def test_workspace_reuse_does_not_leak_between_blocks():
                          *workspaces(M, T, "cuda", hidden=HID, ffn=FFN))
     torch.cuda.synchronize()
     assert torch.equal(y_shared, y_fresh)
+
+
+def test_fused_ffn_block_equals_separate_kernels():
+    """The block with ffn.net.0.proj's epilogue doing GELU + quantization
+    gives the same bits as GEMM -> GELU kernel -> quantizer."""
+    from mxfp8_w8a8_quantized_b200.workloads import Block, workspaces
+    seed = 12
+    x = synth.activations_device(M, HID, seed, 1000, "cuda")
+    ctx = synth.activations_device(T, HID, seed, 1001, "cuda")
+    blk = Block(seed, 0, "cuda", hidden=HID, ffn=FFN)
+    y_fused = blk.forward(x, ctx, *workspaces(M, T, "cuda", hidden=HID, ffn=FFN), fuse_ffn=True)
+    y_sep = blk.forward(x, ctx, *workspaces(M, T, "cuda", hidden=HID, ffn=FFN), fuse_ffn=False)
+    torch.cuda.synchronize()
+    assert torch.equal(y_fused, y_sep)
