@@ -49,8 +49,11 @@ def parse(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOADS[0], choices=WORKLOADS)
     ap.add_argument("--unfused", action="store_true",
-                    help="chained workloads: ffn.net.0.proj writes BF16 and GELU + quantization run as "
-                         "separate kernels (default: fused into its epilogue)")
+                    help="chained workloads: separate q/k/v (and text k/v) GEMMs, and ffn.net.0.proj writes "
+                         "BF16 with GELU + quantization as separate kernels (default: fused)")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture one step as a CUDA graph and time its replays (per-kernel times then "
+                         "come from 3 eager steps)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -331,22 +334,28 @@ class BlocksWorkload(LinearWorkload):
 
     def config(self):
         return {"M": self.M, "text_tokens": self.T, "blocks": self.nblocks, "hidden": self.K, "ffn": self.N,
+                "projections": "fused qkv (N=15360) and text kv (N=10240)" if self.fused else "separate",
                 "ffn0_epilogue": "gelu + quantize fused" if self.fused else "bf16 out; gelu, quantize separate"}
 
-    def _per_block(self):
+    def _launches(self):
+        """The GEMM launches of one block as (rows, K, N, quantized_out) and
+        the stand-alone quantizations as (rows, K)."""
         from mxfp8_w8a8_quantized_b200 import synth
-        fl, qb, gb = 0.0, 0.0, 0.0
-        for name, K, N, kind in synth.block_linears():
-            rows = self.M if kind == "video" else self.T
-            fl += 2.0 * rows * K * N
-            gb += _gemm_bytes(rows, K, N, quantized_out=self.fused and name == "ffn.net.0.proj")
-        # stand-alone quantizations: x (shared by q/k/v), v1, o1, ctx (shared
-        # by k/v), q2, o2, and the GELU output unless fused
-        quants = [(self.M, self.K)] * 5 + [(self.T, self.K)]
-        if not self.fused:
-            quants.append((self.M, self.N))
-        for rows, K in quants:
-            qb += _quant_bytes(rows, K)
+        H, F, M, T = self.K, self.N, self.M, self.T
+        if self.fused:   # fused QKV / KV projections, GELU + quantize in ffn.net.0.proj
+            gemms = [(M, H, 3 * H, False), (M, H, H, False), (M, H, H, False), (T, H, 2 * H, False),
+                     (M, H, H, False), (M, H, F, True), (M, F, H, False)]
+            quants = [(M, H)] * 5 + [(T, H)]
+        else:
+            gemms = [(M if kind == "video" else T, K, N, False) for _, K, N, kind in synth.block_linears()]
+            quants = [(M, H)] * 5 + [(T, H), (M, F)]
+        return gemms, quants
+
+    def _per_block(self):
+        gemms, quants = self._launches()
+        fl = sum(2.0 * r * K * N for r, K, N, _ in gemms)
+        gb = sum(_gemm_bytes(r, K, N, quantized_out=q) for r, K, N, q in gemms)
+        qb = sum(_quant_bytes(r, K) for r, K in quants)
         return fl, qb, gb
 
     def flops(self):
@@ -368,12 +377,13 @@ class BlocksWorkload(LinearWorkload):
         self.blocks = [Block(s, b, dev) for b in range(self.nblocks)]
         self.wa, self.wb = workspaces(self.M, self.T, dev)
         self.y = None
-        self.launches = self.nblocks * (16 if self.fused else 18)
+        gemms, quants = self._launches()
+        self.launches = self.nblocks * (len(gemms) + len(quants) + (0 if self.fused else 1))
 
     def _run(self, T, x):
         y = x
         for blk in self.blocks:
-            y = blk.forward(y, self.ctx, self.wa, self.wb, fuse_ffn=self.fused, timer=T)
+            y = blk.forward(y, self.ctx, self.wa, self.wb, fuse_qkv=self.fused, fuse_ffn=self.fused, timer=T)
         return y
 
     def step(self, T):
@@ -429,15 +439,22 @@ def run_ours(args, ranks, dev):
         raise RuntimeError("kernel reported a pipeline timeout during warm-up")
 
     steps = args.steps
+    graph = None
+    if args.graph:
+        from mxfp8_w8a8_quantized_b200.workloads import StepGraph
+        graph = StepGraph(lambda: wl.step(T))   # T is off: no events inside the graph
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    T.on = True
+    T.on = graph is None
     ranks.barrier()
     torch.cuda.synchronize()
     with ClockSampler(dev.index or 0) as clk:
         for i in range(steps):
             flush.zero_()                      # L2 flushed between timed steps
             ev[i][0].record(stream)
-            wl.step(T)
+            if graph is not None:
+                graph.replay()
+            else:
+                wl.step(T)
             ev[i][1].record(stream)
         torch.cuda.synchronize()
     ranks.barrier()
@@ -447,6 +464,16 @@ def run_ours(args, ranks, dev):
     total_ms = ranks.max(sum(step_ms))
     ms_per_step = total_ms / steps
     value = ranks.world * wl.flops() * steps / (total_ms * 1e-3) / 1e12
+    kernel_steps = steps
+    if graph is not None:
+        # per-kernel device times come from a few eager steps after the timed
+        # graph replays (events cannot sit between a graph's kernels)
+        kernel_steps = min(steps, 3)
+        T.on = True
+        for _ in range(kernel_steps):
+            flush.zero_()
+            wl.step(T)
+        torch.cuda.synchronize()
 
     hbm, bf16_burst, bf16_sustained, peak_src = load_peaks()
     # a single linear is a kernel timed on its own (burst peak); the chained
@@ -456,8 +483,8 @@ def run_ours(args, ranks, dev):
     tot = T.totals()
     g_n, g_ms = tot["gemm"]
     q_n, q_ms = tot["quant"]
-    gemm_tflops = wl.flops() * steps / (g_ms * 1e-3) / 1e12
-    quant_gbs = wl.quant_bytes() * steps / (q_ms * 1e-3) / 1e9
+    gemm_tflops = wl.flops() * kernel_steps / (g_ms * 1e-3) / 1e12
+    quant_gbs = wl.quant_bytes() * kernel_steps / (q_ms * 1e-3) / 1e9
     out = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -474,6 +501,7 @@ def run_ours(args, ranks, dev):
                 "N(0,0.01) f16 bias)",
         "config": dict(workload=wl.name, desc=wl.desc, **wl.config(),
                        l2="flushed between timed steps (256 MiB write outside the step events)",
+                       launch="one CUDA graph per step" if graph is not None else "eager launches",
                        parallelism=f"replicas x{ranks.world}" if ranks.world > 1 else "single GPU"),
         "roofline": {"bound": "tensor", "kernel": "mxfp8_gemm_kernel",
                      "achieved": round(gemm_tflops, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
@@ -481,17 +509,17 @@ def run_ours(args, ranks, dev):
                      "peak_source": f"{peak_src} bf16 {kind} x {FP8_OVER_BF16} (nominal FP8/BF16 ratio)",
                      "traffic": load_traffic(wl.name),
                      "algorithmic_bytes_per_step": round(wl.gemm_bytes()),
-                     "launches_per_step": g_n // steps, "avg_launch_ms": round(g_ms / g_n, 4)},
+                     "launches_per_step": g_n // kernel_steps, "avg_launch_ms": round(g_ms / g_n, 4)},
         "quant": {"kernel": "mx_quantize_kernel", "achieved_gbs": round(quant_gbs, 1), "peak_gbs": hbm,
                   "frac": round(quant_gbs / hbm, 4), "peak_source": f"{peak_src} copy",
-                  "bytes_per_step": wl.quant_bytes(), "launches_per_step": q_n // steps,
+                  "bytes_per_step": wl.quant_bytes(), "launches_per_step": q_n // kernel_steps,
                   "avg_launch_ms": round(q_ms / q_n, 4)},
         "gpu_launches": wl.launches * steps,
         "clocks": clk.summary(),
     }
     if "gelu" in tot:
         n, ms = tot["gelu"]
-        out["gelu"] = {"launches_per_step": n // steps, "avg_launch_ms": round(ms / n, 4)}
+        out["gelu"] = {"launches_per_step": n // kernel_steps, "avg_launch_ms": round(ms / n, 4)}
     if not args.no_e2e:
         out["e2e"] = run_e2e(args, wl, ranks, dev)
     return out

@@ -95,14 +95,20 @@ def linear_workspace_bytes(M: int, K: int) -> int:
 
 
 def quantize(x: torch.Tensor, layout: int = SF_TCGEN05, codes=None, scales=None):
-    """BF16 [M, K] -> (E4M3 codes uint8 [M, K], E8M0 scales uint8 [bytes])."""
-    _cuda(x, "x", torch.bfloat16)
+    """BF16 [M, K] -> (E4M3 codes uint8 [M, K], E8M0 scales uint8 [bytes]).
+    x may be a row-strided view (unit column stride, row stride >= K), e.g.
+    a column slice of a fused projection's output."""
+    if not x.is_cuda or x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D BF16 CUDA tensor")
     M, K = x.shape
+    ldx = x.stride(0) if M > 1 else K
+    if x.stride(1) != 1 or ldx < K:
+        raise ValueError("x must have unit column stride and row stride >= K")
     if codes is None:
         codes = torch.empty((M, K), dtype=torch.uint8, device=x.device)
     if scales is None:
         scales = torch.empty(max(scale_bytes(M, K, layout), 1), dtype=torch.uint8, device=x.device)
-    _check(_lib.mxfp8_quantize(_ptr(x), M, K, K, _ptr(codes), _ptr(scales), layout, _stream()),
+    _check(_lib.mxfp8_quantize(_ptr(x), M, K, ldx, _ptr(codes), _ptr(scales), layout, _stream()),
            "mxfp8_quantize")
     return codes, scales
 

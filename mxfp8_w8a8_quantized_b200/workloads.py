@@ -8,16 +8,21 @@ ffn.net.2; the pages do not give the dataflow between them, so attention is
 replaced by stand-ins that keep every shape):
 
     x  [M, 5120] video tokens          ctx [512, 5120] text tokens
-    q1, k1, v1 = attn1.to_q/k/v(x)      one quantization of x shared by all three
+    q1, k1, v1 = attn1.to_q/k/v(x)      one quantization of x shared by all three;
+                                        one GEMM with N = 15360 (fused QKV projection)
     o1 = attn1.to_out(v1)               self-attention stand-in: identity map, output = V
     q2 = attn2.to_q(o1)
-    k2, v2 = attn2.to_k/v(ctx)          one quantization of ctx shared by both
+    k2, v2 = attn2.to_k/v(ctx)          one quantization of ctx shared by both;
+                                        one GEMM with N = 10240
     o2 = attn2.to_out(q2)               cross-attention stand-in: output = the queries
     f  = ffn.net.0.proj(o2)             [M, 13824]
     g  = GELU_tanh(f)                   in place
     y  = ffn.net.2(g)                   [M, 5120]  -> next block's x
 
 Every linear quantizes its BF16 input dynamically (MXFP8) before the GEMM.
+The fused projections (fuse_qkv, the default) run the concatenated weights
+of q/k/v (and of attn2's k/v) as one GEMM; the outputs are column slices of
+one buffer and every element is computed exactly as by the separate GEMMs.
 With fuse_ffn (the default), ffn.net.0.proj's epilogue applies the GELU and
 quantizes for ffn.net.2 itself (mxfp8_gemm_quantize_out): f and g are never
 written, and the result is bit-identical to the separate kernels.
@@ -38,6 +43,23 @@ class QLinear:
 
     def __init__(self, wq, ws, bias, K, N):
         self.wq, self.ws, self.bias, self.K, self.N = wq, ws, bias, K, N
+
+    @classmethod
+    def concat(cls, parts):
+        """One linear whose output rows are those of `parts` in order (the
+        weights of a fused projection).  Returns (fused, views): `views` are
+        linears over slices of the fused storage, in place of `parts`.  Needs
+        every N % 128 == 0, so that each part's scale atoms are whole."""
+        K = parts[0].K
+        assert all(p.K == K and p.N % 128 == 0 for p in parts)
+        fused = cls(torch.cat([p.wq for p in parts]), torch.cat([p.ws for p in parts]),
+                    torch.cat([p.bias for p in parts]), K, sum(p.N for p in parts))
+        views, r, sb = [], 0, 0
+        for p in parts:
+            nsb = mxfp8.scale_bytes(p.N, K)
+            views.append(cls(fused.wq[r: r + p.N], fused.ws[sb: sb + nsb], fused.bias[r: r + p.N], K, p.N))
+            r, sb = r + p.N, sb + nsb
+        return fused, views
 
     @classmethod
     def random(cls, K, N, seed, index, device):
@@ -82,22 +104,35 @@ class Block:
         width = {synth.HIDDEN: hidden, synth.FFN: ffn}
         for i, (name, K, N, _) in enumerate(synth.block_linears()):
             self.lin[name] = QLinear.random(width[K], width[N], seed, 10 * block_index + i, device)
+        L = self.lin
+        self.qkv, (L["attn1.to_q"], L["attn1.to_k"], L["attn1.to_v"]) = QLinear.concat(
+            [L["attn1.to_q"], L["attn1.to_k"], L["attn1.to_v"]])
+        self.kv2, (L["attn2.to_k"], L["attn2.to_v"]) = QLinear.concat([L["attn2.to_k"], L["attn2.to_v"]])
 
-    def forward(self, x, ctx, ws_a, ws_b, keep=False, fuse_ffn=True, timer=None):
+    def forward(self, x, ctx, ws_a, ws_b, keep=False, fuse_qkv=True, fuse_ffn=True, timer=None):
         """x [M, hidden], ctx [T, hidden] BF16.  ws_a / ws_b: two Workspaces
         (two live quantized activations at most).  Returns y, plus every
         intermediate when keep=True (g only without fuse_ffn)."""
         L = self.lin
         T = timer or _call
+        H = L["attn1.to_q"].N
         xq, xs = T("quant", ws_a.quantize, x)
-        q1 = T("gemm", L["attn1.to_q"], xq, xs)
-        k1 = T("gemm", L["attn1.to_k"], xq, xs)
-        v1 = T("gemm", L["attn1.to_v"], xq, xs)
+        if fuse_qkv:
+            qkv = T("gemm", self.qkv, xq, xs)
+            q1, k1, v1 = qkv[:, :H], qkv[:, H: 2 * H], qkv[:, 2 * H:]
+        else:
+            q1 = T("gemm", L["attn1.to_q"], xq, xs)
+            k1 = T("gemm", L["attn1.to_k"], xq, xs)
+            v1 = T("gemm", L["attn1.to_v"], xq, xs)
         o1 = T("gemm", L["attn1.to_out"], *T("quant", ws_b.quantize, v1))
         q2 = T("gemm", L["attn2.to_q"], *T("quant", ws_a.quantize, o1))
         cq, cs = T("quant", ws_b.quantize, ctx)
-        k2 = T("gemm", L["attn2.to_k"], cq, cs)
-        v2 = T("gemm", L["attn2.to_v"], cq, cs)
+        if fuse_qkv:
+            kv2 = T("gemm", self.kv2, cq, cs)
+            k2, v2 = kv2[:, :H], kv2[:, H:]
+        else:
+            k2 = T("gemm", L["attn2.to_k"], cq, cs)
+            v2 = T("gemm", L["attn2.to_v"], cq, cs)
         o2 = T("gemm", L["attn2.to_out"], *T("quant", ws_a.quantize, q2))
         oq, os_ = T("quant", ws_b.quantize, o2)
         g = None
@@ -115,6 +150,25 @@ class Block:
 
 def _call(kind, fn, *args, **kw):
     return fn(*args, **kw)
+
+
+class StepGraph:
+    """A step (any function of no arguments that only launches work on the
+    current stream, into buffers that stay alive) captured once as a CUDA
+    graph and replayed: one launch for the whole step instead of one per
+    kernel.  The first run happens outside the capture, so that every
+    kernel's one-time set-up is done before capturing."""
+
+    def __init__(self, fn):
+        fn()
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.out = fn()
+
+    def replay(self):
+        self.graph.replay()
+        return self.out
 
 
 def workspaces(M, T, device, hidden=synth.HIDDEN, ffn=synth.FFN):

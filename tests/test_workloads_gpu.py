@@ -79,3 +79,47 @@ def test_fused_ffn_block_equals_separate_kernels():
     y_sep = blk.forward(x, ctx, *workspaces(M, T, "cuda", hidden=HID, ffn=FFN), fuse_ffn=False)
     torch.cuda.synchronize()
     assert torch.equal(y_fused, y_sep)
+
+
+def test_fused_projections_equal_separate_gemms():
+    """q/k/v as one N = 3 hidden GEMM (and attn2's k/v as one): the same
+    bits as the separate GEMMs, for every intermediate and the output."""
+    from mxfp8_w8a8_quantized_b200.workloads import Block, workspaces
+    seed = 13
+    x = synth.activations_device(M, HID, seed, 1000, "cuda")
+    ctx = synth.activations_device(T, HID, seed, 1001, "cuda")
+    blk = Block(seed, 0, "cuda", hidden=HID, ffn=FFN)
+    y_f, mid_f = blk.forward(x, ctx, *workspaces(M, T, "cuda", hidden=HID, ffn=FFN), keep=True, fuse_qkv=True)
+    y_s, mid_s = blk.forward(x, ctx, *workspaces(M, T, "cuda", hidden=HID, ffn=FFN), keep=True, fuse_qkv=False)
+    torch.cuda.synchronize()
+    assert torch.equal(y_f, y_s)
+    for k in ("q1", "k1", "v1", "o1", "q2", "k2", "v2", "o2"):
+        assert torch.equal(mid_f[k], mid_s[k]), k
+
+
+def test_step_graph_replay_equals_eager():
+    """Two blocks captured as one CUDA graph: replays give the eager result,
+    also after the input buffer's contents change."""
+    from mxfp8_w8a8_quantized_b200.workloads import Block, StepGraph, workspaces
+    seed = 14
+    x = synth.activations_device(M, HID, seed, 1000, "cuda")
+    ctx = synth.activations_device(T, HID, seed, 1001, "cuda")
+    blocks = [Block(seed, b, "cuda", hidden=HID, ffn=FFN) for b in range(2)]
+    wa, wb = workspaces(M, T, "cuda", hidden=HID, ffn=FFN)
+
+    def step():
+        y = x
+        for blk in blocks:
+            y = blk.forward(y, ctx, wa, wb)
+        return y
+
+    eager = step().clone()
+    g = StepGraph(step)
+    assert torch.equal(g.replay(), eager)
+    x.copy_(synth.activations_device(M, HID, seed, 2000, "cuda"))
+    eager2 = step().clone()
+    assert torch.equal(g.replay(), eager2)
+    assert not torch.equal(eager, eager2)
+    torch.cuda.synchronize()
+    from mxfp8_w8a8_quantized_b200 import mxfp8
+    assert mxfp8.device_status() == 0
