@@ -51,6 +51,9 @@ def lib():
         L.orc_linear_f32acc.argtypes = [P, P, I64, I64, P, P, I64, P, P, I64, P, I64, P]
         L.orc_bf16_rne_array.argtypes = [P, I64, P]
         L.orc_gelu_tanh_bf16.argtypes = [P, I64, P]
+        L.orc_quantize_rowwise_bf16.argtypes = [P, I64, I64, I64, P, P]
+        L.orc_quantize_rowwise_f32.argtypes = [P, I64, I64, P, P]
+        L.orc_linear_rowwise.argtypes = [P, P, I64, I64, P, P, I64, P, P, I64, P, I64, P]
         L.orc_num_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -205,3 +208,44 @@ def linear_f32acc(xq, xs, wq, ws, bias_bits=None, rows=None, cols=None):
 
 def num_threads():
     return int(lib().orc_num_threads())
+
+
+# ------------------------------------------------------ per-channel FP8
+def quantize_rowwise_bf16(x_bits):
+    """BF16 bits [M, K] -> (E4M3 codes [M, K], FP32 scales [M]); one scale
+    amax / 448 per row, codes E4M3(x / s) (binary32 divisions)."""
+    x = _c(x_bits, np.uint16)
+    M, K = x.shape
+    codes = np.empty((M, K), dtype=np.uint8)
+    scales = np.empty(M, dtype=np.float32)
+    lib().orc_quantize_rowwise_bf16(_ptr(x), M, K, K, _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def quantize_rowwise_f32(w):
+    """FP32 [N, K] -> (E4M3 codes [N, K], FP32 scales [N]), one per output channel."""
+    w = _c(w, np.float32)
+    N, K = w.shape
+    codes = np.empty((N, K), dtype=np.uint8)
+    scales = np.empty(N, dtype=np.float32)
+    lib().orc_quantize_rowwise_f32(_ptr(w), N, K, _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def linear_rowwise(xq, sx, wq, sw, bias_bits=None, rows=None, cols=None):
+    """Exact per-channel FP8 linear for the selected rows / cols (FP64)."""
+    xq = _c(xq, np.uint8)
+    wq = _c(wq, np.uint8)
+    sx = _c(sx, np.float32)
+    sw = _c(sw, np.float32)
+    M, K = xq.shape
+    N = wq.shape[0]
+    r = None if rows is None else _c(rows, np.int64)
+    c = None if cols is None else _c(cols, np.int64)
+    nr = M if r is None else len(r)
+    nc = N if c is None else len(c)
+    b = None if bias_bits is None else _c(bias_bits, np.uint16)
+    y = np.empty((nr, nc), dtype=np.float64)
+    lib().orc_linear_rowwise(_ptr(xq), _ptr(sx), M, K, _ptr(wq), _ptr(sw), N, _ptr(b), _ptr(r), nr, _ptr(c), nc,
+                             _ptr(y))
+    return y

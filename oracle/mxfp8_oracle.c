@@ -37,6 +37,22 @@
  *    output is that value rounded to nearest-even.
  *  - GELU between the two FFN linears is the tanh form
  *    0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))).
+ *
+ * Per-channel FP8 (the "fp8-vllm" / "fp8-sgl" modes of [LQ] SS "Quantization
+ * Modes": FP8 channel-symmetric weights, FP8 channel-dynamic symmetric
+ * activations; SS "MiniMax-H3 FP8 with FP16 Accumulation": activations use
+ * dynamic row-wise quantization with scale = max(abs(x)) / qmax; qmax is 448
+ * with FP32 accumulation, SS "MiniMax-H3 Video VAE Encoder Conv3D"; the
+ * LightX2V Wan2.2 FP8 checkpoints keep "per-output-channel FP32 scales",
+ * page "Wan2.2 I2V A14B, four-step 720p: native LightX2V FP8 and NVFP4",
+ * SS "Conversion and compatibility"):
+ *  - one FP32 scale per activation row (token) and per weight row (output
+ *    channel): s = amax / 448, a binary32 division of the row's largest
+ *    magnitude (the pages give the scales as FP32);
+ *  - codes are E4M3(x / s) with x / s a binary32 division, rounded to nearest
+ *    even and saturating at 448 as above; a row of zeros has s = 0 and codes
+ *    of +-0;
+ *  - Y = s_x[m] s_w[n] sum_k xq[m,k] wq[n,k] + bias[n], exact (FP64 here).
  */
 #include <math.h>
 #include <stddef.h>
@@ -395,6 +411,96 @@ void orc_gelu_tanh_bf16(const uint16_t *x, int64_t n, uint16_t *y)
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n; ++i)
         y[i] = orc_bf16_rne(orc_gelu_tanh(orc_bf16_decode(x[i])));
+}
+
+/* ------------------------------------------------------------------ */
+/* Per-channel FP8: one FP32 scale per row                             */
+/* ------------------------------------------------------------------ */
+
+/*
+ * One row of K binary32 values -> E4M3 codes and the row's FP32 scale
+ * s = amax / 448.  Both the scale and the quotients x / s are binary32
+ * divisions (IEEE, round to nearest even); the quotient then goes to the
+ * E4M3 encoder, which rounds it to nearest even and saturates at 448.
+ */
+static void quantize_row_f32(const float *x, int64_t K, uint8_t *codes, float *scale)
+{
+    float amax = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+        float a = fabsf(x[k]);
+        if (a > amax)
+            amax = a;
+    }
+    volatile float s = amax / 448.0f; /* binary32 division */
+    *scale = s;
+    for (int64_t k = 0; k < K; ++k) {
+        if (s == 0.0f) {
+            codes[k] = orc_e4m3_encode(x[k]); /* +-0 */
+        } else {
+            volatile float q = x[k] / s;  /* binary32 division */
+            codes[k] = orc_e4m3_encode((double)q);
+        }
+    }
+}
+
+/* BF16 activations [rows, K] (row stride ldx) -> codes [rows, K], FP32 scales [rows]. */
+void orc_quantize_rowwise_bf16(const uint16_t *x, int64_t rows, int64_t K, int64_t ldx, uint8_t *codes,
+                               float *scales)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        float *row = (float *)malloc((size_t)K * sizeof(float));
+        if (!row)
+            continue;
+        for (int64_t k = 0; k < K; ++k)
+            row[k] = (float)orc_bf16_decode(x[r * ldx + k]);
+        quantize_row_f32(row, K, codes + r * K, scales + r);
+        free(row);
+    }
+}
+
+/* FP32 weights [rows, K] -> codes [rows, K], FP32 scales [rows] (one per output channel). */
+void orc_quantize_rowwise_f32(const float *w, int64_t rows, int64_t K, uint8_t *codes, float *scales)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        quantize_row_f32(w + r * K, K, codes + r * K, scales + r);
+}
+
+/*
+ * Per-channel FP8 linear: Y[i, j] = sx[m] sw[n] sum_k dec(xq[m,k]) dec(wq[n,k])
+ * + bias[n] (m = rows[i], n = cols[j]), exact in FP64.
+ */
+void orc_linear_rowwise(const uint8_t *xq, const float *sx, int64_t M, int64_t K, const uint8_t *wq,
+                        const float *sw, int64_t N, const uint16_t *bias, const int64_t *rows, int64_t nr,
+                        const int64_t *cols, int64_t nc, double *Y)
+{
+    (void)M;
+    (void)N;
+    double *wd = (double *)malloc((size_t)nc * (size_t)K * sizeof(double));
+    if (!wd)
+        return;
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < nc; ++j) {
+        int64_t n = cols ? cols[j] : j;
+        for (int64_t k = 0; k < K; ++k)
+            wd[j * K + k] = orc_e4m3_decode(wq[n * K + k]);
+    }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < nr; ++i) {
+        int64_t r = rows ? rows[i] : i;
+        for (int64_t j = 0; j < nc; ++j) {
+            int64_t n = cols ? cols[j] : j;
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += orc_e4m3_decode(xq[r * K + k]) * wd[j * K + k];
+            acc = acc * (double)sx[r] * (double)sw[n];
+            if (bias)
+                acc += orc_f16_decode(bias[n]);
+            Y[i * nc + j] = acc;
+        }
+    }
+    free(wd);
 }
 
 /* Threads an OpenMP parallel region uses (1 without OpenMP). */

@@ -2,7 +2,9 @@
 
 Each case edits one line of a copy of oracle/mxfp8_oracle.c (an off-by-one
 scale exponent, ties to odd, a transposed weight index, a dropped bias, a
-wrong scale index, overflow to NaN instead of saturation, a lost sign), builds the copy and
+wrong scale index, overflow to NaN instead of saturation, a lost sign; for the
+per-channel FP8 functions a wrong qmax, an amax over part of the row, a zero
+row divided by its zero scale, a dropped weight scale), builds the copy and
 runs the pins against it; the pins must fail.  The real oracle is untouched.
 """
 import os
@@ -25,7 +27,14 @@ MUTATIONS = {
                         "if (a >= e4m3_mag[0x7E])\n        return sign | 0x7F;"),
     "sign_lost": ("return sign | (uint8_t)pick;", "return (uint8_t)pick;"),
     "subnormal_scale_wrong": ("mag = ldexp((double)m, -9);", "mag = ldexp((double)m, -10);"),
+    # per-channel FP8
+    "rowwise_qmax_wrong": ("volatile float s = amax / 448.0f;", "volatile float s = amax / 447.0f;"),
+    "rowwise_amax_half_row": ("for (int64_t k = 0; k < K; ++k) {\n        float a = fabsf(x[k]);",
+                              "for (int64_t k = 0; k < K / 2; ++k) {\n        float a = fabsf(x[k]);"),
+    "rowwise_zero_row_divides": ("if (s == 0.0f) {", "if (0) {"),
+    "rowwise_weight_scale_dropped": ("acc = acc * (double)sx[r] * (double)sw[n];", "acc = acc * (double)sx[r];"),
 }
+PIN_FILES = ["test_oracle_pins.py", "test_oracle_pins_rowwise.py"]
 
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
@@ -41,7 +50,7 @@ def test_pins_catch_planted_mistake(name):
         subprocess.run(["gcc", "-O1", "-std=c11", "-D_DEFAULT_SOURCE", "-fPIC", "-shared",
                         "-fopenmp", "-ffp-contract=off", "-o", so, c, "-lm"], check=True)
         env = dict(os.environ, ORACLE_LIB=so, OMP_NUM_THREADS="2")
-        r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                            os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+        r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider"]
+                           + [os.path.join(ROOT, "tests", f) for f in PIN_FILES],
                            cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
         assert r.returncode != 0, f"pins did not catch mutation {name}:\n{r.stdout[-2000:]}"
