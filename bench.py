@@ -51,6 +51,8 @@ def parse(argv=None):
     ap.add_argument("--unfused", action="store_true",
                     help="chained workloads: separate q/k/v (and text k/v) GEMMs, and ffn.net.0.proj writes "
                          "BF16 with GELU + quantization as separate kernels (default: fused)")
+    ap.add_argument("--scheme", choices=["mxfp8", "fp8rowwise"], default="mxfp8",
+                    help="quantization scheme of the single-linear workloads (default: MXFP8)")
     ap.add_argument("--graph", action="store_true",
                     help="capture one step as a CUDA graph and time its replays (per-kernel times then "
                          "come from 3 eager steps)")
@@ -199,9 +201,14 @@ class LinearWorkload:
     """One quantized linear: Y = BF16(MXFP8(X) MXFP8(W)^T + b)."""
 
     long_step = False
+    scheme = "mxfp8"
 
     def __init__(self, name, M, K, N, seed, desc):
         self.name, self.M, self.K, self.N, self.seed, self.desc = name, M, K, N, seed, desc
+
+    @property
+    def profile_key(self):
+        return self.name if self.scheme == "mxfp8" else f"{self.name}_{self.scheme}"
 
     def config(self):
         return {"M": self.M, "K": self.K, "N": self.N}
@@ -256,6 +263,49 @@ def _gemm_bytes(M, K, N, quantized_out=False):
 def _quant_bytes(M, K):
     """Algorithmic HBM bytes of one activation quantization."""
     return M * K * 3 + M * K // 32
+
+
+class FP8RowwiseLinearWorkload(LinearWorkload):
+    """One per-channel FP8 linear: FP32 scale per token (dynamic, amax / 448)
+    and per output channel; Y = BF16(sx sw (Xq . Wq^T) + b)."""
+
+    scheme = "fp8rowwise"
+
+    def config(self):
+        return {"M": self.M, "K": self.K, "N": self.N,
+                "scheme": "per-channel FP8 (E4M3, FP32 scale per token and per output channel)"}
+
+    def quant_bytes(self):
+        return self.M * self.K * 3 + 4 * self.M
+
+    def gemm_bytes(self):
+        M, K, N = self.M, self.K, self.N
+        return M * K + N * K + 4 * M + 4 * N + 2 * M * N + 2 * N
+
+    def setup(self, dev):
+        from mxfp8_w8a8_quantized_b200 import mxfp8, synth
+        self.mx = mxfp8
+        M, K, N, s = self.M, self.K, self.N, self.seed
+        self.x = synth.activations_device(M, K, s, 0, dev)
+        w = synth.weights_device(N, K, s, 0, dev)
+        self.b = synth.bias_device(N, s, 0, dev)
+        self.wq, self.ws = mxfp8.fp8rw_quantize_weight(w)   # offline weight quantization
+        del w
+        self.xq = torch.empty((M, K), dtype=torch.uint8, device=dev)
+        self.xs = torch.empty(M, dtype=torch.float32, device=dev)
+        self.y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        self.launches = 2
+
+    def step(self, T):
+        mx = self.mx
+        T("quant", mx.fp8rw_quantize, self.x, codes=self.xq, scales=self.xs)
+        T("gemm", mx.fp8rw_gemm, self.xq, self.xs, self.wq, self.ws, self.b, out=self.y)
+
+    def e2e_step(self, x_dev, y_dev, ws):
+        self.mx.fp8rw_linear(x_dev, self.wq, self.ws, self.b, out=y_dev, workspace=ws)
+
+    def e2e_workspace(self, dev):
+        return torch.empty(self.mx.fp8rw_linear_workspace_bytes(self.M, self.K), dtype=torch.uint8, device=dev)
 
 
 class FFNPairWorkload(LinearWorkload):
@@ -399,8 +449,13 @@ class BlocksWorkload(LinearWorkload):
         return None
 
 
-def make_workload(name, fused=True):
+def make_workload(name, fused=True, scheme="mxfp8"):
     from mxfp8_w8a8_quantized_b200 import synth
+    if scheme == "fp8rowwise":
+        wl = make_workload(name)
+        if type(wl) is not LinearWorkload:
+            raise ValueError("the per-channel FP8 scheme is measured on the single-linear workloads")
+        return FP8RowwiseLinearWorkload(wl.name, wl.M, wl.K, wl.N, wl.seed, wl.desc)
     H, F = synth.HIDDEN, synth.FFN
     M1, M2, T = synth.TOKENS_480P, synth.TOKENS_832x1104, synth.TEXT_TOKENS
     if name == "c0_small":
@@ -425,7 +480,7 @@ def make_workload(name, fused=True):
 
 # ---------------------------------------------------------------- our arm
 def run_ours(args, ranks, dev):
-    wl = make_workload(args.workload, fused=not args.unfused)
+    wl = make_workload(args.workload, fused=not args.unfused, scheme=args.scheme)
     wl.setup(dev)
     stream = torch.cuda.current_stream(dev)
     mx = wl.mx
@@ -507,7 +562,7 @@ def run_ours(args, ranks, dev):
                      "achieved": round(gemm_tflops, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
                      "frac": round(gemm_tflops / fp8_peak, 4),
                      "peak_source": f"{peak_src} bf16 {kind} x {FP8_OVER_BF16} (nominal FP8/BF16 ratio)",
-                     "traffic": load_traffic(wl.name),
+                     "traffic": load_traffic(wl.profile_key),
                      "algorithmic_bytes_per_step": round(wl.gemm_bytes()),
                      "launches_per_step": g_n // kernel_steps, "avg_launch_ms": round(g_ms / g_n, 4)},
         "quant": {"kernel": "mx_quantize_kernel", "achieved_gbs": round(quant_gbs, 1), "peak_gbs": hbm,
@@ -588,15 +643,21 @@ def oracle_sample(wl, rows):
     x = synth.activations(rows, wl.K, wl.seed, index=100)
     w = synth.weights(wl.N, wl.K, wl.seed, index=100)
     b = synth.bias(wl.N, wl.seed, index=100)
-    wq, ws = oracle.quantize_f32(w.numpy())
+    if wl.scheme == "fp8rowwise":
+        wq, ws = oracle.quantize_rowwise_f32(w.numpy())
+    else:
+        wq, ws = oracle.quantize_f32(w.numpy())
     xb = x.view(torch.int16).numpy().view(np.uint16)
     bb = b.view(torch.int16).numpy().view(np.uint16)
-    return xb, wq, ws, bb
+    return xb, wq, ws, bb, wl.scheme
 
 
-def oracle_step(xb, wq, ws, bb):
+def oracle_step(xb, wq, ws, bb, scheme):
     """One step of the oracle on the sample: quantize the rows, FP64 linear."""
     import oracle
+    if scheme == "fp8rowwise":
+        xq, xs = oracle.quantize_rowwise_bf16(xb)
+        return oracle.linear_rowwise(xq, xs, wq, ws, bb)
     xq, xs = oracle.quantize_bf16(xb)
     return oracle.linear(xq, xs, wq, ws, bb)
 
@@ -605,9 +666,9 @@ def size_sample(wl, target_s, max_rows=None):
     """Rows whose oracle step takes about target_s seconds."""
     rows, dt = 4, 0.0
     for _ in range(6):
-        xb, wq, ws, bb = oracle_sample(wl, rows)
+        sample = oracle_sample(wl, rows)
         t0 = time.perf_counter()
-        oracle_step(xb, wq, ws, bb)
+        oracle_step(*sample)
         dt = time.perf_counter() - t0
         if dt >= 0.5 * target_s:
             break
@@ -617,15 +678,79 @@ def size_sample(wl, target_s, max_rows=None):
     return rows
 
 
+def chain_oracle_sample(wl):
+    """A bounded sample of a chained workload for the oracle: video-token
+    rows through the FFN pair, or through one block (its text-token linears
+    on a proportional number of text rows, at least one).  Weights are
+    quantized by the oracle here, outside any timed region.  Returns
+    make(rows) -> (run, flops)."""
+    import numpy as np
+
+    import oracle
+    from mxfp8_w8a8_quantized_b200 import synth
+
+    def lin(K, N, i):
+        wq, ws = oracle.quantize_f32(synth.weights(N, K, wl.seed, index=200 + i).numpy())
+        b = synth.bias(N, wl.seed, index=200 + i).view(torch.int16).numpy().view(np.uint16)
+        return wq, ws, b
+
+    def apply(x_bits, w):
+        xq, xs = oracle.quantize_bf16(x_bits)
+        return oracle.bf16_rne(oracle.linear(xq, xs, *w))
+
+    def rows_of(n, K, index):
+        return synth.activations(n, K, wl.seed, index=index).view(torch.int16).numpy().view(np.uint16)
+
+    H, F = wl.K, wl.N
+    if isinstance(wl, FFNPairWorkload):
+        l0, l2 = lin(H, F, 0), lin(F, H, 1)
+
+        def make(rows):
+            x = rows_of(rows, H, 300)
+            return (lambda: apply(oracle.gelu_tanh_bf16(apply(x, l0)), l2)), 2 * 2.0 * rows * H * F
+        return make
+    L = {name: lin(K, N, i) for i, (name, K, N, _) in enumerate(synth.block_linears())}
+
+    def make(rows):
+        trows = max(1, round(rows * wl.T / wl.M))
+        x, ctx = rows_of(rows, H, 300), rows_of(trows, H, 301)
+
+        def run():
+            for name in ("attn1.to_q", "attn1.to_k"):
+                apply(x, L[name])
+            o1 = apply(apply(x, L["attn1.to_v"]), L["attn1.to_out"])
+            o2 = apply(apply(o1, L["attn2.to_q"]), L["attn2.to_out"])
+            for name in ("attn2.to_k", "attn2.to_v"):
+                apply(ctx, L[name])
+            return apply(oracle.gelu_tanh_bf16(apply(o2, L["ffn.net.0.proj"])), L["ffn.net.2"])
+        return run, 2.0 * (rows * (6 * H * H + 2 * H * F) + trows * 2 * H * H)
+    return make
+
+
 def cpu_baseline(wl, target_s):
     import oracle
-    if not isinstance(wl, LinearWorkload) or type(wl) is not LinearWorkload:
-        return {"value": None, "unit": "TFLOP/s", "kind": "oracle", "cores": oracle.num_threads(),
-                "sample": "not measured for chained workloads"}
+    if type(wl) not in (LinearWorkload, FP8RowwiseLinearWorkload):
+        # chained: grow the row sample until one pass takes about target_s
+        make = chain_oracle_sample(wl)
+        rows = 2
+        for _ in range(8):
+            run, fl = make(rows)
+            t0 = time.perf_counter()
+            run()
+            dt = time.perf_counter() - t0
+            if dt >= 0.5 * target_s or rows >= wl.M:
+                break
+            rows = int(min(wl.M, max(rows * 2, rows * 0.9 * target_s / max(dt, 1e-3))))
+        what = "the FFN pair" if isinstance(wl, FFNPairWorkload) else "one block (text linears on a proportional " \
+            "number of text rows)"
+        return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                "kind": "oracle",
+                "sample": f"{rows} video-token rows through {what}: quantize + FP64 linear per linear, GELU; "
+                          f"weights quantized outside the timed region; {dt:.1f} s"}
     rows = size_sample(wl, target_s)
-    xb, wq, ws, bb = oracle_sample(wl, rows)
+    sample = oracle_sample(wl, rows)
     t0 = time.perf_counter()
-    oracle_step(xb, wq, ws, bb)
+    oracle_step(*sample)
     dt = time.perf_counter() - t0
     return {"value": round(2.0 * rows * wl.N * wl.K / dt / 1e12, 6), "unit": "TFLOP/s",
             "cores": oracle.num_threads(), "kind": "oracle",
@@ -636,21 +761,20 @@ def cpu_baseline(wl, target_s):
 def run_reference(args, ranks):
     """The oracle as the reference arm: CPU, rank 0 only."""
     import oracle
-    wl = make_workload(args.workload)
-    if type(wl) is not LinearWorkload:
-        wl = make_workload("c1_q_proj_480p") if args.workload == "c1_q_proj_480p" else \
-            LinearWorkload(wl.name, wl.M, wl.K, wl.K, wl.seed, wl.desc + " (first linear only)")
+    wl = make_workload(args.workload, scheme=args.scheme)
+    if type(wl) not in (LinearWorkload, FP8RowwiseLinearWorkload):
+        wl = LinearWorkload(wl.name, wl.M, wl.K, wl.K, wl.seed, wl.desc + " (first linear only)")
     if ranks.rank != 0:
         return None
     budget = args.reference_seconds  # warm-up + timed steps together
     n_steps = args.steps + args.warmup
     rows = size_sample(wl, budget / n_steps)
-    xb, wq, ws, bb = oracle_sample(wl, rows)
+    sample = oracle_sample(wl, rows)
     for _ in range(args.warmup):
-        oracle_step(xb, wq, ws, bb)
+        oracle_step(*sample)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(xb, wq, ws, bb)
+        oracle_step(*sample)
     dt = time.perf_counter() - t0
     value = 2.0 * rows * wl.N * wl.K * args.steps / dt / 1e12
     sample = f"{rows} of {wl.M} rows per step (quantize + FP64 linear over all {wl.N} columns, K={wl.K})"
@@ -691,7 +815,8 @@ def main(argv=None):
         out = run_ours(args, ranks, dev)
         if ranks.rank == 0:
             if ranks.world == 1 and not args.no_cpu_baseline:
-                out["cpu_baseline"] = cpu_baseline(make_workload(args.workload), args.cpu_seconds)
+                out["cpu_baseline"] = cpu_baseline(make_workload(args.workload, scheme=args.scheme),
+                                                   args.cpu_seconds)
             print(json.dumps(out), flush=True)
     finally:
         ranks.close()

@@ -16,7 +16,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmxfp8.so")
 
-SOURCES = ["mxfp8_quant.cu", "mxfp8_gemm.cu", "mxfp8_capi.cu", "mxfp8_noalloc.cu"]
+PUBLIC_HEADERS = ["mxfp8.h", "fp8_rowwise.h"]
+SOURCES = ["mxfp8_quant.cu", "mxfp8_gemm.cu", "mxfp8_capi.cu", "mxfp8_noalloc.cu", "fp8_rowwise.cu"]
 HEADERS = ["ptx.cuh", "mx_element.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -31,13 +32,13 @@ def nvcc() -> str:
 
 def _inputs():
     return ([os.path.join(CSRC, s) for s in SOURCES + HEADERS]
-            + [os.path.join(INCLUDE, "mxfp8.h"), os.path.abspath(__file__)])
+            + [os.path.join(INCLUDE, h) for h in PUBLIC_HEADERS] + [os.path.abspath(__file__)])
 
 
 def source_sha() -> str:
     """Hash of the kernel sources; ties a profile summary to one build."""
     h = hashlib.sha256()
-    for p in [os.path.join(CSRC, s) for s in SOURCES + HEADERS] + [os.path.join(INCLUDE, "mxfp8.h")]:
+    for p in [os.path.join(CSRC, s) for s in SOURCES + HEADERS] + [os.path.join(INCLUDE, h) for h in PUBLIC_HEADERS]:
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "fp8_rowwise.h"
 #include "mxfp8.h"
 
 namespace mx {
@@ -15,6 +16,8 @@ int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void
                 const void *bias, void *Y, int epi, void *S, cudaStream_t stream, unsigned long long timeout_ns,
                 cudaError_t *err);
 cudaError_t read_and_clear_status(unsigned int *out);
+cudaError_t launch_fp8_rowwise_quantize(const void *X, bool f32_in, int64_t M, int64_t K, int64_t ldx, uint8_t *Q,
+                                        float *S, cudaStream_t stream);
 } // namespace mx
 
 namespace {
@@ -212,6 +215,89 @@ mxfp8_status mxfp8_gelu_tanh_bf16(const void *X, void *Y, int64_t n, mxfp8_strea
     if (!aligned(X, 16) || !aligned(Y, 16))
         return MXFP8_ERR_ALIGN;
     return from_cuda(mx::launch_gelu(X, Y, n, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+/* ---------------------------------------------------- per-channel FP8 */
+
+mxfp8_status fp8rw_quantize_bf16(const void *X, int64_t M, int64_t K, int64_t ldx, void *codes, float *scales,
+                                 mxfp8_stream_t stream)
+{
+    if (M < 0 || K <= 0 || ldx < K)
+        return MXFP8_ERR_ARG;
+    if (M == 0)
+        return MXFP8_OK;
+    if (!X || !codes || !scales)
+        return MXFP8_ERR_ARG;
+    if (K % 8 != 0 || K > FP8RW_MAX_K || M > kMaxRows)
+        return MXFP8_ERR_SHAPE;
+    if (!aligned(X, 16) || (ldx * 2) % 16 != 0 || !aligned(codes, 8) || !aligned(scales, 4))
+        return MXFP8_ERR_ALIGN;
+    return from_cuda(mx::launch_fp8_rowwise_quantize(X, false, M, K, ldx, static_cast<uint8_t *>(codes), scales,
+                                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mxfp8_status fp8rw_quantize_weight_f32(const float *W, int64_t N, int64_t K, void *Wq, float *Wscale,
+                                       mxfp8_stream_t stream)
+{
+    if (N < 0 || K <= 0)
+        return MXFP8_ERR_ARG;
+    if (N == 0)
+        return MXFP8_OK;
+    if (!W || !Wq || !Wscale)
+        return MXFP8_ERR_ARG;
+    if (K % 4 != 0 || K > FP8RW_MAX_K || N > kMaxRows)
+        return MXFP8_ERR_SHAPE;
+    if (!aligned(W, 16) || !aligned(Wq, 4) || !aligned(Wscale, 4))
+        return MXFP8_ERR_ALIGN;
+    return from_cuda(mx::launch_fp8_rowwise_quantize(W, true, N, K, K, static_cast<uint8_t *>(Wq), Wscale,
+                                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mxfp8_status fp8rw_gemm(const void *Xq, const float *Xscale, int64_t M, int64_t K, const void *Wq,
+                        const float *Wscale, int64_t N, const void *bias, void *Y, mxfp8_stream_t stream)
+{
+    mxfp8_status st = gemm_args(Xq, Xscale, M, K, Wq, Wscale, N, bias, Y);
+    if (st != MXFP8_OK || M == 0)
+        return st;
+    cudaError_t e;
+    int r = mx::launch_gemm(Xq, Xscale, M, K, Wq, Wscale, N, bias, Y, 3, nullptr,
+                            reinterpret_cast<cudaStream_t>(stream), kWaitLimitNs, &e);
+    if (r == 1)
+        return MXFP8_ERR_CUDA;
+    return r == 0 ? MXFP8_OK : from_cuda(e);
+}
+
+size_t fp8rw_linear_workspace_bytes(int64_t M, int64_t K)
+{
+    if (M < 0 || K <= 0)
+        return 0;
+    return round_up((size_t)M * (size_t)K, 256) + (size_t)M * sizeof(float);
+}
+
+mxfp8_status fp8rw_linear(const void *X, int64_t M, int64_t K, const void *Wq, const float *Wscale, int64_t N,
+                          const void *bias, void *Y, void *workspace, size_t ws_bytes, mxfp8_stream_t stream)
+{
+    if (M < 0 || K <= 0 || N <= 0)
+        return MXFP8_ERR_ARG;
+    if (M == 0)
+        return MXFP8_OK;
+    if (!X || !workspace)
+        return MXFP8_ERR_ARG;
+    if (K % 128 != 0 || K > FP8RW_MAX_K)
+        return MXFP8_ERR_SHAPE;
+    if (!aligned(workspace, 256) || !aligned(X, 16))
+        return MXFP8_ERR_ALIGN;
+    if (ws_bytes < fp8rw_linear_workspace_bytes(M, K))
+        return MXFP8_ERR_ARG;
+    uint8_t *codes = static_cast<uint8_t *>(workspace);
+    float *scales = reinterpret_cast<float *>(codes + round_up((size_t)M * (size_t)K, 256));
+    mxfp8_status st = gemm_args(codes, scales, M, K, Wq, Wscale, N, bias, Y);
+    if (st != MXFP8_OK)
+        return st;
+    st = fp8rw_quantize_bf16(X, M, K, K, codes, scales, stream);
+    if (st != MXFP8_OK)
+        return st;
+    return fp8rw_gemm(codes, scales, M, K, Wq, Wscale, N, bias, Y, stream);
 }
 
 mxfp8_status mxfp8_device_status(mxfp8_stream_t stream)

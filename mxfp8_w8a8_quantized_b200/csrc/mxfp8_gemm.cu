@@ -93,6 +93,7 @@ enum EpiMode : int {
     EPI_BF16 = 0,       /* Y = BF16(acc + bias) */
     EPI_QUANT = 1,      /* MXFP8 codes + scales of BF16(acc + bias) for the next linear */
     EPI_QUANT_GELU = 2, /* MXFP8 codes + scales of BF16(GELU(BF16(acc + bias))) */
+    EPI_ROWWISE = 3,    /* per-channel FP8: no block scales; Y = BF16(acc sx[m] sw[n] + bias) */
 };
 
 template <bool PAIR>
@@ -133,6 +134,8 @@ struct GemmParams {
     const __half *bias;   /* [N] or null */
     __nv_bfloat16 *Y;     /* [M, N] (EPI_BF16) */
     uint8_t *S;           /* output scales, tensor-core layout of [M, N] (quantizing modes) */
+    const float *sx;      /* [M] row scales (EPI_ROWWISE) */
+    const float *sw;      /* [N] column scales (EPI_ROWWISE) */
     int M, N, K;
     int m_pad;            /* M rounded up to 128: rows that own scale bytes */
     int sf_kgroups;       /* N / 128: scale atoms per 128 output rows */
@@ -212,6 +215,64 @@ __device__ __forceinline__ void epilogue_bf16(const uint32_t (&acc)[128], const 
                 __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(acc[a]) + b[2 * j],
                                                          __uint_as_float(acc[a + 1]) + b[2 * j + 1]);
                 o[j] = *reinterpret_cast<uint32_t *>(&v);
+            }
+            st_shared_v4(rowbase + ((((uint32_t)j8) ^ swz) << 4), o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmap_y, colc, row0, buf);
+            bulk_commit_group();
+        }
+    }
+}
+
+/* Per-channel FP8 epilogue: Y = BF16(acc sx[row] sw[col] + bias), staged and
+ * stored like the BF16 epilogue.  The thread's row scale is one load; the
+ * column scales come 8 at a time with the bias. */
+__device__ __forceinline__ void epilogue_rowwise(const uint32_t (&acc)[128], const GemmParams &p,
+                                                 const CUtensorMap *tmap_y, int row0, int col0, int lane,
+                                                 uint32_t buf, uint32_t rowbase, uint32_t swz)
+{
+    const int row = row0 + lane;
+    const float sxr = row < p.M ? __ldg(p.sx + row) : 0.0f;
+    const f32x2 sx2 = f2_pack(sxr, sxr);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const int colc = col0 + 32 * c;
+        if (row0 >= p.M || colc >= p.N) /* whole box outside Y: nothing to store */
+            continue;
+        if (lane == 0)
+            bulk_wait_group_read0(); /* previous box has left the buffer */
+        __syncwarp();
+#pragma unroll
+        for (int j8 = 0; j8 < 4; ++j8) {
+            const int col = colc + 8 * j8;
+            float b[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            float w[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (col < p.N) {
+                const uint4 w0 = __ldg(reinterpret_cast<const uint4 *>(p.sw + col));
+                const uint4 w1 = __ldg(reinterpret_cast<const uint4 *>(p.sw + col + 4));
+                w[0] = __uint_as_float(w0.x), w[1] = __uint_as_float(w0.y), w[2] = __uint_as_float(w0.z);
+                w[3] = __uint_as_float(w0.w), w[4] = __uint_as_float(w1.x), w[5] = __uint_as_float(w1.y);
+                w[6] = __uint_as_float(w1.z), w[7] = __uint_as_float(w1.w);
+                if (p.bias) {
+                    const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(p.bias + col));
+                    const __half2 *bh = reinterpret_cast<const __half2 *>(&bv);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 f2 = __half22float2(bh[j]);
+                        b[2 * j] = f2.x;
+                        b[2 * j + 1] = f2.y;
+                    }
+                }
+            }
+            uint32_t o[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int a = 32 * c + 8 * j8 + 2 * j;
+                const f32x2 t = f2_mul(f2_pack(__uint_as_float(acc[a]), __uint_as_float(acc[a + 1])), sx2);
+                o[j] = f32x2_to_bf16x2(f2_fma(t, f2_pack(w[2 * j], w[2 * j + 1]), f2_pack(b[2 * j], b[2 * j + 1])));
             }
             st_shared_v4(rowbase + ((((uint32_t)j8) ^ swz) << 4), o[0], o[1], o[2], o[3]);
         }
@@ -338,6 +399,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                       const __grid_constant__ CUtensorMap tmap_y, const GemmParams p)
 {
     using C = Cfg<PAIR>;
+    constexpr bool BS = EPI != EPI_ROWWISE; /* MXFP8 block scales (else per-channel FP8) */
+    constexpr uint32_t STAGE_TX = BS ? C::STAGE_TX : (C::A_BYTES + C::B_BYTES) * (PAIR ? 2u : 1u);
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -395,8 +458,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (lane == 0) {
             prefetch_tmap(&tmap_a);
             prefetch_tmap(&tmap_b);
-            prefetch_tmap(&tmap_sfa);
-            prefetch_tmap(&tmap_sfb);
+            if constexpr (BS) {
+                prefetch_tmap(&tmap_sfa);
+                prefetch_tmap(&tmap_sfb);
+            }
             uint32_t it = 0;
             bool ok = true;
             for (int t = tile0; ok && t < num_tiles; t += tstep) {
@@ -414,7 +479,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     }
                     const uint32_t full = bar_full + 8 * s;
                     if (rank == 0)
-                        mbar_arrive_expect_tx(full, C::STAGE_TX);
+                        mbar_arrive_expect_tx(full, STAGE_TX);
                     const uint32_t dA = sbase + C::OFF_A + s * C::A_BYTES;
                     const uint32_t dB = sbase + C::OFF_B + s * C::B_BYTES;
                     const uint32_t dSA = sbase + C::OFF_SFA + s * C::SFA_BYTES;
@@ -444,13 +509,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         const uint32_t lead = mapa_shared(full, 0u);
                         tma_load_2d_pair(dA, &tmap_a, kb * BK, rowA, lead);
                         tma_load_2d_pair(dB, &tmap_b, kb * BK, rowB, lead);
-                        tma_load_3d_pair(dSA, &tmap_sfa, 0, kb, rbA, lead);
-                        tma_load_3d_pair(dSB, &tmap_sfb, 0, kb, rbB, lead);
+                        if constexpr (BS) {
+                            tma_load_3d_pair(dSA, &tmap_sfa, 0, kb, rbA, lead);
+                            tma_load_3d_pair(dSB, &tmap_sfb, 0, kb, rbB, lead);
+                        }
                     } else {
                         tma_load_2d(dA, &tmap_a, kb * BK, rowA, full);
                         tma_load_2d(dB, &tmap_b, kb * BK, rowB, full);
-                        tma_load_3d(dSA, &tmap_sfa, 0, kb, rbA, full);
-                        tma_load_3d(dSB, &tmap_sfb, 0, kb, rbB, full);
+                        if constexpr (BS) {
+                            tma_load_3d(dSA, &tmap_sfa, 0, kb, rbA, full);
+                            tma_load_3d(dSB, &tmap_sfb, 0, kb, rbB, full);
+                        }
                     }
                 }
             }
@@ -458,7 +527,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     } else if (warp == 1) {
         /* ------------------------------------------------ MMA issuer */
         if (lane == 0 && rank == 0) {
-            const uint32_t idesc = idesc_mxf8_e4m3(C::TILE_M, C::TILE_N);
+            const uint32_t idesc = BS ? idesc_mxf8_e4m3(C::TILE_M, C::TILE_N) : idesc_f8_e4m3(C::TILE_M, C::TILE_N);
             uint32_t it = 0, tl = 0;
             bool ok = true, any = false;
             for (int t = tile0; ok && t < num_tiles; t += tstep, ++tl) {
@@ -470,7 +539,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const uint32_t s = it % C::STAGES, ph = (it / C::STAGES) & 1u;
                     if (!wait_bounded(bar_full + 8 * s, ph, lim, abort_flag) ||
-                        (PAIR && !wait_bounded(bar_sffull + 8 * s, ph, lim, abort_flag))) {
+                        (PAIR && BS && !wait_bounded(bar_sffull + 8 * s, ph, lim, abort_flag))) {
                         ok = false;
                         break;
                     }
@@ -481,7 +550,25 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     const uint32_t sfb_s = sbase + C::OFF_SFB + s * C::SFB_BYTES;
                     const uint64_t adesc = desc_kmajor_sw128(sbase + C::OFF_A + s * C::A_BYTES);
                     const uint64_t bdesc = desc_kmajor_sw128(sbase + C::OFF_B + s * C::B_BYTES);
-                    if constexpr (PAIR) {
+                    if constexpr (!BS) {
+                        (void)tsfa;
+                        (void)tsfb;
+                        (void)sfa_s;
+                        (void)sfb_s;
+#pragma unroll
+                        for (int k = 0; k < BK / 32; ++k) {
+                            if constexpr (PAIR)
+                                tc_mma_f8_pair(tmem + ACC_COL, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k),
+                                               idesc, (kb | k) != 0);
+                            else
+                                tc_mma_f8(tmem + ACC_COL, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc,
+                                          (kb | k) != 0);
+                        }
+                        if constexpr (PAIR)
+                            tc_commit_pair(bar_empty + 8 * s, (uint16_t)0x3);
+                        else
+                            tc_commit(bar_empty + 8 * s);
+                    } else if constexpr (PAIR) {
                         /* scales were copied to TMEM by the scale warp */
                         (void)sfa_s;
                         (void)sfb_s;
@@ -529,7 +616,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         /* The pair-wide tcgen05.cp holds up the thread that issues it, so it
          * is issued here, one stage at a time, and the MMA thread only waits
          * for its completion (sf_full), never for the copy itself. */
-        if (PAIR && lane == 0 && rank == 0) {
+        if (PAIR && BS && lane == 0 && rank == 0) {
             uint32_t it = 0;
             for (int t = tile0; t < num_tiles; t += tstep) {
                 bool ok = true;
@@ -586,6 +673,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const uint32_t swz = ((uint32_t)lane >> 1) & 3u;
             if constexpr (EPI == EPI_BF16)
                 epilogue_bf16(acc, p, &tmap_y, row0, col0, lane, buf, rowbase, swz);
+            else if constexpr (EPI == EPI_ROWWISE)
+                epilogue_rowwise(acc, p, &tmap_y, row0, col0, lane, buf, rowbase, swz);
             else
                 epilogue_quantize<EPI == EPI_QUANT_GELU>(acc, p, &tmap_y, row0, col0, lane, buf, rowbase, swz);
         }
@@ -696,7 +785,7 @@ struct DevInfo {
     int sms = 148;
     bool pair_checked = false;
     int max_pair_clusters = 0;   /* 0: pairs unavailable */
-    bool attr[2][3] = {};        /* [PAIR][EPI]: shared-memory attribute set */
+    bool attr[2][4] = {};        /* [PAIR][EPI]: shared-memory attribute set */
 };
 static DevInfo g_dev[64];
 
@@ -794,6 +883,8 @@ static cudaError_t launch_mode(DevInfo *d, int epi, const CUtensorMap &ma, const
         return launch_variant<PAIR, EPI_QUANT>(d, ma, mb, msa, msb, my, p, grid, stream);
     case EPI_QUANT_GELU:
         return launch_variant<PAIR, EPI_QUANT_GELU>(d, ma, mb, msa, msb, my, p, grid, stream);
+    case EPI_ROWWISE:
+        return launch_variant<PAIR, EPI_ROWWISE>(d, ma, mb, msa, msb, my, p, grid, stream);
     default:
         return launch_variant<PAIR, EPI_BF16>(d, ma, mb, msa, msb, my, p, grid, stream);
     }
@@ -813,13 +904,15 @@ static bool pair_enabled()
 /*
  * epi = 0: Y is BF16 [M, N], S unused.  epi = 1 / 2: Y receives E4M3 codes
  * [M, N] and S the tensor-core scales of [M, N] (2: GELU before the
- * quantization); N % 128 == 0.
+ * quantization); N % 128 == 0.  epi = 3 (per-channel FP8): Xs / Ws are FP32
+ * row scales [M] / [N], Y is BF16 [M, N].
  * Returns 0 ok, 1 tensor-map failure, 2 CUDA error (in *err).
  */
 int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void *Wq, const void *Ws, int64_t N,
                 const void *bias, void *Y, int epi, void *S, cudaStream_t stream, unsigned long long timeout_ns,
                 cudaError_t *err)
 {
+    const bool bs = epi != EPI_ROWWISE;
     *err = cudaSuccess;
     if (M == 0)
         return 0;
@@ -837,14 +930,23 @@ int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void
 
     const uint32_t b_rows = pair ? Cfg<true>::B_ROWS : Cfg<false>::B_ROWS;
     CUtensorMap ma, mb, msa, msb, my;
-    const bool out_ok = epi == EPI_BF16 ? make_output_map(&my, Y, M, N) : make_codes_out_map(&my, Y, M, N);
-    if (!make_operand_map(&ma, Xq, M, K, 128) || !make_operand_map(&mb, Wq, N, K, b_rows) ||
-        !make_scale_map(&msa, Xs, M, K, 1) || !make_scale_map(&msb, Ws, N, K, 2) || !out_ok)
+    const bool out_ok = (epi == EPI_BF16 || epi == EPI_ROWWISE) ? make_output_map(&my, Y, M, N)
+                                                                 : make_codes_out_map(&my, Y, M, N);
+    if (!make_operand_map(&ma, Xq, M, K, 128) || !make_operand_map(&mb, Wq, N, K, b_rows) || !out_ok)
         return 1;
+    if (bs) {
+        if (!make_scale_map(&msa, Xs, M, K, 1) || !make_scale_map(&msb, Ws, N, K, 2))
+            return 1;
+    } else {
+        msa = ma; /* not read without block scales */
+        msb = mb;
+    }
     GemmParams p;
     p.bias = static_cast<const __half *>(bias);
     p.Y = static_cast<__nv_bfloat16 *>(Y);
     p.S = static_cast<uint8_t *>(S);
+    p.sx = bs ? nullptr : static_cast<const float *>(Xs);
+    p.sw = bs ? nullptr : static_cast<const float *>(Ws);
     p.M = (int)M;
     p.N = (int)N;
     p.K = (int)K;

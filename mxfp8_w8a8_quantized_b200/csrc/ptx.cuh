@@ -303,6 +303,29 @@ __device__ __forceinline__ void tc_mma_mxf8_pair(uint32_t tacc, uint64_t adesc, 
         : "memory");
 }
 
+/* D(tmem) (+)= A(smem) . B(smem)^T, E4M3 x E4M3 without block scales, 32-wide
+ * K, over the CTA pair (same operand split as tc_mma_mxf8_pair). */
+__device__ __forceinline__ void tc_mma_f8_pair(uint32_t tacc, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tacc),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_f8(uint32_t tacc, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tacc),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 /* ------------------------------------------------- operand descriptors */
 /*
  * Shared-memory matrix descriptor, K-major operand written by TMA with the
@@ -341,6 +364,15 @@ __device__ __forceinline__ uint64_t desc_sf_32x16(uint32_t saddr)
 __host__ __device__ constexpr uint32_t idesc_mxf8_e4m3(int M, int N)
 {
     return (0u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24);
+}
+/*
+ * Instruction descriptor of kind::f8f6f4 without block scaling: FP32
+ * accumulator (1 at [4,6)), A and B E4M3 (0 at [7,10) and [10,13)), both
+ * K-major, N >> 3 at [17,23), M >> 4 at [24,29).
+ */
+__host__ __device__ constexpr uint32_t idesc_f8_e4m3(int M, int N)
+{
+    return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 __host__ __device__ constexpr uint32_t idesc_with_sf_id(uint32_t idesc, uint32_t id)
 {

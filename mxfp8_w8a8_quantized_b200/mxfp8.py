@@ -44,6 +44,16 @@ _lib.mxfp8_linear_noalloc.argtypes = [_P, _I64, _I64, _P, _P, _I64, _P, _P, _P]
 _lib.mxfp8_linear_noalloc.restype = ctypes.c_int
 _lib.mxfp8_gemm_quantize_out.argtypes = [_P, _P, _I64, _I64, _P, _P, _I64, _P, ctypes.c_int, _P, _P, _P]
 _lib.mxfp8_gemm_quantize_out.restype = ctypes.c_int
+_lib.fp8rw_quantize_bf16.argtypes = [_P, _I64, _I64, _I64, _P, _P, _P]
+_lib.fp8rw_quantize_bf16.restype = ctypes.c_int
+_lib.fp8rw_quantize_weight_f32.argtypes = [_P, _I64, _I64, _P, _P, _P]
+_lib.fp8rw_quantize_weight_f32.restype = ctypes.c_int
+_lib.fp8rw_gemm.argtypes = [_P, _P, _I64, _I64, _P, _P, _I64, _P, _P, _P]
+_lib.fp8rw_gemm.restype = ctypes.c_int
+_lib.fp8rw_linear_workspace_bytes.argtypes = [_I64, _I64]
+_lib.fp8rw_linear_workspace_bytes.restype = _SZ
+_lib.fp8rw_linear.argtypes = [_P, _I64, _I64, _P, _P, _I64, _P, _P, _P, _SZ, _P]
+_lib.fp8rw_linear.restype = ctypes.c_int
 _lib.mxfp8_device_status.argtypes = [_P]
 _lib.mxfp8_device_status.restype = ctypes.c_int
 
@@ -55,7 +65,9 @@ ACT_GELU_TANH = 1
 EXPORTS = ("mxfp8_status_str", "mxfp8_scale_bytes", "mxfp8_quantize", "mxfp8_quantize_weight_f32",
            "mxfp8_linear_workspace_bytes", "mxfp8_linear", "mxfp8_gemm_prequant",
            "mxfp8_gelu_tanh_bf16", "mxfp8_device_status", "mxfp8_linear_noalloc",
-           "mxfp8_gemm_quantize_out")
+           "mxfp8_gemm_quantize_out",
+           "fp8rw_quantize_bf16", "fp8rw_quantize_weight_f32", "fp8rw_gemm", "fp8rw_linear_workspace_bytes",
+           "fp8rw_linear")
 
 
 class MXFP8Error(RuntimeError):
@@ -188,6 +200,65 @@ def gelu_tanh(x: torch.Tensor, out=None):
     if out is None:
         out = torch.empty_like(x)
     _check(_lib.mxfp8_gelu_tanh_bf16(_ptr(x), _ptr(out), x.numel(), _stream()), "mxfp8_gelu_tanh_bf16")
+    return out
+
+
+# ------------------------------------------------------ per-channel FP8
+def fp8rw_quantize(x: torch.Tensor, codes=None, scales=None):
+    """BF16 [M, K] -> (E4M3 codes uint8 [M, K], FP32 scales [M]): one scale
+    amax / 448 per row (token).  x may be a row-strided view."""
+    if not x.is_cuda or x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D BF16 CUDA tensor")
+    M, K = x.shape
+    ldx = x.stride(0) if M > 1 else K
+    if x.stride(1) != 1 or ldx < K:
+        raise ValueError("x must have unit column stride and row stride >= K")
+    if codes is None:
+        codes = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(_lib.fp8rw_quantize_bf16(_ptr(x), M, K, ldx, _ptr(codes), _ptr(scales), _stream()),
+           "fp8rw_quantize_bf16")
+    return codes, scales
+
+
+def fp8rw_quantize_weight(w: torch.Tensor):
+    """FP32 [N, K] -> (E4M3 codes uint8 [N, K], FP32 scales [N]), one per output channel."""
+    _cuda(w, "w", torch.float32)
+    N, K = w.shape
+    codes = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    scales = torch.empty(N, dtype=torch.float32, device=w.device)
+    _check(_lib.fp8rw_quantize_weight_f32(_ptr(w), N, K, _ptr(codes), _ptr(scales), _stream()),
+           "fp8rw_quantize_weight_f32")
+    return codes, scales
+
+
+def fp8rw_gemm(xq, xscale, wq, wscale, bias=None, out=None):
+    """Y = BF16(sx sw (Xq . Wq^T) + bias) from per-channel FP8 operands."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    _check(_lib.fp8rw_gemm(_ptr(xq), _ptr(xscale), M, K, _ptr(wq), _ptr(wscale), N, _ptr(bias), _ptr(out),
+                           _stream()), "fp8rw_gemm")
+    return out
+
+
+def fp8rw_linear_workspace_bytes(M: int, K: int) -> int:
+    return int(_lib.fp8rw_linear_workspace_bytes(M, K))
+
+
+def fp8rw_linear(x: torch.Tensor, wq, wscale, bias=None, out=None, workspace=None):
+    """The per-channel FP8 layer: quantize x per token, then fp8rw_gemm."""
+    _cuda(x, "x", torch.bfloat16)
+    M, K = x.shape
+    N = wq.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(max(fp8rw_linear_workspace_bytes(M, K), 256), dtype=torch.uint8, device=x.device)
+    _check(_lib.fp8rw_linear(_ptr(x), M, K, _ptr(wq), _ptr(wscale), N, _ptr(bias), _ptr(out), _ptr(workspace),
+                             workspace.numel(), _stream()), "fp8rw_linear")
     return out
 
 

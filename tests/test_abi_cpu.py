@@ -1,4 +1,4 @@
-"""The C-ABI library loads and exports every symbol include/mxfp8.h declares;
+"""The C-ABI library loads and exports every symbol include/*.h declares;
 host-side argument checks reject bad calls before anything is launched.
 No GPU needed: none of these calls reaches the device."""
 import ctypes
@@ -8,13 +8,19 @@ import re
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "mxfp8.h")
+INCLUDE = os.path.join(ROOT, "include")
+PREFIXES = ("mxfp8_", "fp8rw_")
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(mxfp8_[a-z0-9_]+)\s*\(", text)))
+    names = set()
+    for h in sorted(os.listdir(INCLUDE)):
+        if not h.endswith(".h"):
+            continue
+        text = open(os.path.join(INCLUDE, h)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"\b((?:%s)[a-z0-9_]+)\s*\(" % "|".join(PREFIXES), text))
+    return sorted(names)
 
 
 @pytest.fixture(scope="module")
@@ -34,7 +40,7 @@ def test_header_declares_the_boundary():
 
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
-        assert hasattr(lib, name), f"{name} declared in include/mxfp8.h but not exported"
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
 
 
 def test_binding_exports_match_header():
@@ -112,6 +118,34 @@ def test_argument_checks_return_before_launch(lib):
     assert L.mxfp8_gelu_tanh_bf16(FAKE, FAKE, 12, None) == SHAPE
     assert L.mxfp8_gelu_tanh_bf16(FAKE, FAKE + 4, 16, None) == ALIGN
     assert L.mxfp8_gelu_tanh_bf16(FAKE, FAKE, 0, None) == 0
+
+
+def test_fp8_rowwise_argument_checks_return_before_launch(lib):
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    lib.fp8rw_quantize_bf16.argtypes = [P, I64, I64, I64, P, P, P]
+    lib.fp8rw_quantize_weight_f32.argtypes = [P, I64, I64, P, P, P]
+    lib.fp8rw_gemm.argtypes = [P, P, I64, I64, P, P, I64, P, P, P]
+    lib.fp8rw_linear_workspace_bytes.argtypes = [I64, I64]
+    lib.fp8rw_linear_workspace_bytes.restype = ctypes.c_size_t
+    lib.fp8rw_linear.argtypes = [P, I64, I64, P, P, I64, P, P, P, ctypes.c_size_t, P]
+    L = lib
+    ARG, ALIGN, SHAPE = 1, 2, 3
+    assert L.fp8rw_quantize_bf16(FAKE, 4, 60, 60, FAKE, FAKE, None) == SHAPE         # K % 8
+    assert L.fp8rw_quantize_bf16(FAKE, 4, 16392, 16392, FAKE, FAKE, None) == SHAPE   # K > 16384
+    assert L.fp8rw_quantize_bf16(FAKE, 4, 64, 60, FAKE, FAKE, None) == ARG           # ldx < K
+    assert L.fp8rw_quantize_bf16(FAKE, 4, 64, 68, FAKE, FAKE, None) == ALIGN         # row stride
+    assert L.fp8rw_quantize_bf16(FAKE, 4, 64, 64, FAKE, FAKE + 2, None) == ALIGN     # scales
+    assert L.fp8rw_quantize_bf16(None, 4, 64, 64, FAKE, FAKE, None) == ARG
+    assert L.fp8rw_quantize_bf16(FAKE, 0, 64, 64, FAKE, FAKE, None) == 0
+    assert L.fp8rw_quantize_weight_f32(FAKE, 4, 66, FAKE, FAKE, None) == SHAPE      # K % 4
+    assert L.fp8rw_quantize_weight_f32(FAKE + 4, 4, 64, FAKE, FAKE, None) == ALIGN
+    assert L.fp8rw_gemm(FAKE, FAKE, 4, 96, FAKE, FAKE, 16, None, FAKE, None) == SHAPE
+    assert L.fp8rw_gemm(FAKE, FAKE + 4, 4, 128, FAKE, FAKE, 16, None, FAKE, None) == ALIGN
+    assert L.fp8rw_gemm(FAKE, FAKE, 0, 128, FAKE, FAKE, 16, None, FAKE, None) == 0
+    need = L.fp8rw_linear_workspace_bytes(4, 128)
+    assert need == 512 + 16
+    assert L.fp8rw_linear(FAKE, 4, 128, FAKE, FAKE, 16, None, FAKE, FAKE, need - 1, None) == ARG
+    assert L.fp8rw_linear(FAKE, 4, 128, FAKE, FAKE, 16, None, FAKE, FAKE + 16, need, None) == ALIGN
 
 
 def test_product_fails_loudly_without_library(tmp_path, monkeypatch):
