@@ -17,7 +17,8 @@ int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void
                 cudaError_t *err);
 cudaError_t read_and_clear_status(unsigned int *out);
 cudaError_t launch_fp8_rowwise_quantize(const void *X, bool f32_in, int64_t M, int64_t K, int64_t ldx, uint8_t *Q,
-                                        float *S, cudaStream_t stream);
+                                        float *S, cudaStream_t stream, unsigned long long timeout_ns);
+cudaError_t read_and_clear_rw_status(unsigned int *out);
 } // namespace mx
 
 namespace {
@@ -233,7 +234,7 @@ mxfp8_status fp8rw_quantize_bf16(const void *X, int64_t M, int64_t K, int64_t ld
     if (!aligned(X, 16) || (ldx * 2) % 16 != 0 || !aligned(codes, 8) || !aligned(scales, 4))
         return MXFP8_ERR_ALIGN;
     return from_cuda(mx::launch_fp8_rowwise_quantize(X, false, M, K, ldx, static_cast<uint8_t *>(codes), scales,
-                                                     reinterpret_cast<cudaStream_t>(stream)));
+                                                     reinterpret_cast<cudaStream_t>(stream), kWaitLimitNs));
 }
 
 mxfp8_status fp8rw_quantize_weight_f32(const float *W, int64_t N, int64_t K, void *Wq, float *Wscale,
@@ -250,7 +251,7 @@ mxfp8_status fp8rw_quantize_weight_f32(const float *W, int64_t N, int64_t K, voi
     if (!aligned(W, 16) || !aligned(Wq, 4) || !aligned(Wscale, 4))
         return MXFP8_ERR_ALIGN;
     return from_cuda(mx::launch_fp8_rowwise_quantize(W, true, N, K, K, static_cast<uint8_t *>(Wq), Wscale,
-                                                     reinterpret_cast<cudaStream_t>(stream)));
+                                                     reinterpret_cast<cudaStream_t>(stream), kWaitLimitNs));
 }
 
 mxfp8_status fp8rw_gemm(const void *Xq, const float *Xscale, int64_t M, int64_t K, const void *Wq,
@@ -305,10 +306,10 @@ mxfp8_status mxfp8_device_status(mxfp8_stream_t stream)
     cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess)
         return MXFP8_ERR_CUDA;
-    unsigned int word = 0;
-    if (mx::read_and_clear_status(&word) != cudaSuccess)
+    unsigned int word = 0, rw_word = 0;
+    if (mx::read_and_clear_status(&word) != cudaSuccess || mx::read_and_clear_rw_status(&rw_word) != cudaSuccess)
         return MXFP8_ERR_CUDA;
-    return word ? MXFP8_ERR_TIMEOUT : MXFP8_OK;
+    return (word | rw_word) ? MXFP8_ERR_TIMEOUT : MXFP8_OK;
 }
 
 } // extern "C"
