@@ -71,7 +71,12 @@ constexpr int SF_WARP = 2 + EPI_WARPS; /* copies scales to TMEM (CTA-pair varian
 constexpr int GEMM_THREADS = (3 + EPI_WARPS) * 32;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0; /* 256 FP32 columns */
-constexpr int RASTER_GROUP = 8; /* M tiles walked together for L2 reuse */
+/* M tiles walked together (for every N tile) so that their A rows stay in
+ * L2: 8 when the weights fit in L2 alongside them, 16 when the weights are
+ * re-read from DRAM once per group (measured: ffn.net.0.proj 4.6 -> 2.6 GB
+ * of DRAM reads per launch; the Q projection reads least with 8). */
+constexpr int RASTER_SMALL_B = 8, RASTER_LARGE_B = 16;
+constexpr int64_t RASTER_LARGE_B_BYTES = 48ll << 20;
 #ifndef MX_PREFETCH_KB
 #define MX_PREFETCH_KB 0
 #endif
@@ -140,15 +145,16 @@ struct GemmParams {
     int m_pad;            /* M rounded up to 128: rows that own scale bytes */
     int sf_kgroups;       /* N / 128: scale atoms per 128 output rows */
     int num_m, num_n;     /* output tiles */
+    int raster;           /* M tiles per raster group */
     unsigned long long timeout_ns;
 };
 
-__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int &mb, int &nb)
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int raster, int &mb, int &nb)
 {
-    const int per_group = RASTER_GROUP * num_n;
+    const int per_group = raster * num_n;
     const int g = t / per_group;
-    const int first = g * RASTER_GROUP;
-    const int gm = min(RASTER_GROUP, num_m - first);
+    const int first = g * raster;
+    const int gm = min(raster, num_m - first);
     const int r = t - g * per_group;
     mb = first + r % gm;
     nb = r / gm;
@@ -466,7 +472,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             bool ok = true;
             for (int t = tile0; ok && t < num_tiles; t += tstep) {
                 int mb, nb;
-                tile_coords(t, p.num_m, p.num_n, mb, nb);
+                tile_coords(t, p.num_m, p.num_n, p.raster, mb, nb);
                 const int rowA = mb * C::TILE_M + (int)(rank * 128u);
                 const int rowB = nb * C::TILE_N + (int)(rank * C::B_ROWS);
                 const int rbA = rowA / 128;
@@ -496,7 +502,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         if (pt < num_tiles && pkb < KB) {
                             int pmb = mb, pnb = nb;
                             if (pt != t)
-                                tile_coords(pt, p.num_m, p.num_n, pmb, pnb);
+                                tile_coords(pt, p.num_m, p.num_n, p.raster, pmb, pnb);
                             const int pra = pmb * C::TILE_M + (int)(rank * 128u);
                             const int prb = pnb * C::TILE_N + (int)(rank * C::B_ROWS);
                             if (pra < p.M)
@@ -648,7 +654,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         uint32_t tl = 0;
         for (int t = tile0; t < num_tiles; t += tstep, ++tl) {
             int mb, nb;
-            tile_coords(t, p.num_m, p.num_n, mb, nb);
+            tile_coords(t, p.num_m, p.num_n, p.raster, mb, nb);
             /* every lane polls; the vote keeps the warp converged for the
              * .sync.aligned TMEM load and makes the outcome warp-uniform */
             const bool got = wait_bounded(bar_tfull, tl & 1u, lim, abort_flag, SUSPEND_EPI);
@@ -955,6 +961,7 @@ int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void
     const int tile_m = pair ? Cfg<true>::TILE_M : Cfg<false>::TILE_M;
     p.num_m = (int)((M + tile_m - 1) / tile_m);
     p.num_n = (int)((N + 255) / 256);
+    p.raster = N * K > RASTER_LARGE_B_BYTES ? RASTER_LARGE_B : RASTER_SMALL_B;
     p.timeout_ns = timeout_ns;
     const int tiles = p.num_m * p.num_n;
     cudaError_t e;
