@@ -54,6 +54,14 @@ def lib():
         L.orc_quantize_rowwise_bf16.argtypes = [P, I64, I64, I64, P, P]
         L.orc_quantize_rowwise_f32.argtypes = [P, I64, I64, P, P]
         L.orc_linear_rowwise.argtypes = [P, P, I64, I64, P, P, I64, P, P, I64, P, I64, P]
+        L.orc_e2m1_decode.argtypes = [ctypes.c_uint8]
+        L.orc_e2m1_decode.restype = ctypes.c_double
+        L.orc_e2m1_encode.argtypes = [ctypes.c_double]
+        L.orc_e2m1_encode.restype = ctypes.c_uint8
+        L.orc_nvfp4_quantize_bf16.argtypes = [P, I64, I64, I64, ctypes.c_float, P, P]
+        L.orc_nvfp4_dequantize.argtypes = [P, P, I64, I64, ctypes.c_float, P]
+        L.orc_nvfp4_linear.argtypes = [P, P, ctypes.c_float, I64, I64, P, P, ctypes.c_float, I64, P, P, I64, P,
+                                       I64, P]
         L.orc_num_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -249,3 +257,65 @@ def linear_rowwise(xq, sx, wq, sw, bias_bits=None, rows=None, cols=None):
     lib().orc_linear_rowwise(_ptr(xq), _ptr(sx), M, K, _ptr(wq), _ptr(sw), N, _ptr(b), _ptr(r), nr, _ptr(c), nc,
                              _ptr(y))
     return y
+
+
+# ------------------------------------------------------------------ NVFP4
+def e2m1_decode(codes):
+    """E2M1 code(s) (0..15) -> float64 value(s)."""
+    c = np.asarray(codes, dtype=np.uint8)
+    f = np.vectorize(lambda v: lib().orc_e2m1_decode(int(v)), otypes=[np.float64])
+    return f(c)
+
+
+def e2m1_encode(values):
+    """Real value(s) -> nearest E2M1 code(s), ties to even, saturating at 6."""
+    v = np.asarray(values, dtype=np.float64)
+    f = np.vectorize(lambda x: lib().orc_e2m1_encode(float(x)), otypes=[np.uint8])
+    return f(v)
+
+
+def nvfp4_quantize_bf16(x_bits, g):
+    """BF16 bits [M, K] and global scale g -> (packed E2M1 codes [M, K/2],
+    UE4M3 scales [M, K/16])."""
+    x = _c(x_bits, np.uint16)
+    M, K = x.shape
+    codes = np.empty((M, K // 2), dtype=np.uint8)
+    scales = np.empty((M, K // 16), dtype=np.uint8)
+    lib().orc_nvfp4_quantize_bf16(_ptr(x), M, K, K, float(np.float32(g)), _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def nvfp4_dequantize(codes, scales, g):
+    codes = _c(codes, np.uint8)
+    scales = _c(scales, np.uint8)
+    M = codes.shape[0]
+    K = codes.shape[1] * 2
+    out = np.empty((M, K), dtype=np.float64)
+    lib().orc_nvfp4_dequantize(_ptr(codes), _ptr(scales), M, K, float(np.float32(g)), _ptr(out))
+    return out
+
+
+def nvfp4_linear(xq, xs, gx, wq, ws, gw, bias_bits=None, rows=None, cols=None):
+    """Exact NVFP4 linear for the selected rows / cols (FP64)."""
+    xq = _c(xq, np.uint8)
+    xs = _c(xs, np.uint8)
+    wq = _c(wq, np.uint8)
+    ws = _c(ws, np.uint8)
+    M = xq.shape[0]
+    K = xq.shape[1] * 2
+    N = wq.shape[0]
+    r = None if rows is None else _c(rows, np.int64)
+    c = None if cols is None else _c(cols, np.int64)
+    nr = M if r is None else len(r)
+    nc = N if c is None else len(c)
+    b = None if bias_bits is None else _c(bias_bits, np.uint16)
+    y = np.empty((nr, nc), dtype=np.float64)
+    lib().orc_nvfp4_linear(_ptr(xq), _ptr(xs), float(np.float32(gx)), M, K, _ptr(wq), _ptr(ws),
+                           float(np.float32(gw)), N, _ptr(b), _ptr(r), nr, _ptr(c), nc, _ptr(y))
+    return y
+
+
+def nvfp4_global_scale(amax):
+    """The per-tensor global scale 448 * 6 / amax (binary32): the largest
+    block then gets the largest UE4M3 scale."""
+    return np.float32(np.float32(448.0 * 6.0) / np.float32(amax))

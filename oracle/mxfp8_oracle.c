@@ -53,6 +53,23 @@
  *    even and saturating at 448 as above; a row of zeros has s = 0 and codes
  *    of +-0;
  *  - Y = s_x[m] s_w[n] sum_k xq[m,k] wq[n,k] + bias[n], exact (FP64 here).
+ *
+ * NVFP4 (page "Wan2.2 I2V A14B, four-step 720p: native LightX2V FP8 and
+ * NVFP4", SS "Conversion and compatibility": packed E2M1 weights with E4M3
+ * block scales, plus FP32 input_global_scale and alpha fields; weights
+ * enter the quantizer as BF16).  The pages name the fields, not the
+ * arithmetic; readings:
+ *  - E2M1: sign, 2 exponent bits (bias 1), 1 mantissa bit; magnitudes
+ *    0, 0.5, 1, 1.5, 2, 3, 4, 6; nearest, ties to the even mantissa,
+ *    saturating at 6.  Two codes per byte, the lower-index element in the
+ *    low nibble.
+ *  - blocks of 16 consecutive K elements share one scale byte, an E4M3
+ *    value used unsigned (UE4M3); one FP32 global scale g per tensor.
+ *  - per block: s = UE4M3(RN(amax * RN(g / 6))) (nearest even, saturating
+ *    at 448); elements E2M1(RN(x * RN(g / dec(s)))), all in binary32; a
+ *    block whose scale is 0 gets codes +-0.
+ *  - dequantized value q dec(s) / g; the layer Y = alpha sum_k qx sx qw sw
+ *    + bias with alpha = 1 / (g_x g_w), exact here.
  */
 #include <math.h>
 #include <stddef.h>
@@ -499,6 +516,140 @@ void orc_linear_rowwise(const uint8_t *xq, const float *sx, int64_t M, int64_t K
                 acc += orc_f16_decode(bias[n]);
             Y[i * nc + j] = acc;
         }
+    }
+    free(wd);
+}
+
+/* ------------------------------------------------------------------ */
+/* NVFP4: E2M1 elements, UE4M3 scales per 16, FP32 global scale        */
+/* ------------------------------------------------------------------ */
+
+/* E2M1: value of one 4-bit code (bit 3 sign, bits 2-1 exponent, bit 0 mantissa). */
+double orc_e2m1_decode(uint8_t c)
+{
+    int s = (c >> 3) & 1;
+    int E = (c >> 1) & 3;
+    int m = c & 1;
+    double mag = E == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, E - 1);
+    return s ? -mag : mag;
+}
+
+/* Nearest E2M1 code, ties to the even mantissa, magnitudes >= 6 -> 6. */
+uint8_t orc_e2m1_encode(double v)
+{
+    uint8_t sign = signbit(v) ? 8 : 0;
+    double a = fabs(v);
+    if (isnan(v))
+        return 7; /* out of contract: never produced for finite inputs */
+    if (a >= 6.0)
+        return sign | 7; /* saturate (far above 6 the distances below would tie) */
+    int best = 0;
+    for (int c = 1; c < 8; ++c) {
+        double dc = fabs(orc_e2m1_decode((uint8_t)c) - a), db = fabs(orc_e2m1_decode((uint8_t)best) - a);
+        if (dc < db || (dc == db && (c & 1) == 0))
+            best = c;
+    }
+    return sign | (uint8_t)best;
+}
+
+/*
+ * One row of K binary32 values -> K/2 packed E2M1 bytes and K/16 UE4M3 scale
+ * bytes, global scale g (binary32 arithmetic throughout, as read above).
+ */
+static void nvfp4_row(const float *x, int64_t K, float g, uint8_t *codes, uint8_t *scales)
+{
+    volatile float gs = g / 6.0f;
+    for (int64_t b = 0; b < K / 16; ++b) {
+        float amax = 0.0f;
+        for (int j = 0; j < 16; ++j) {
+            float a = fabsf(x[16 * b + j]);
+            if (a > amax)
+                amax = a;
+        }
+        volatile float sf = amax * gs;
+        uint8_t sb = orc_e4m3_encode((double)sf) & 0x7F; /* unsigned use of E4M3 */
+        scales[b] = sb;
+        double ds = orc_e4m3_decode(sb);
+        volatile float mul = ds > 0.0 ? g / (float)ds : 0.0f;
+        for (int j = 0; j < 16; j += 2) {
+            uint8_t lo, hi;
+            if (ds > 0.0) {
+                volatile float q0 = x[16 * b + j] * mul, q1 = x[16 * b + j + 1] * mul;
+                lo = orc_e2m1_encode((double)q0);
+                hi = orc_e2m1_encode((double)q1);
+            } else {
+                lo = orc_e2m1_encode(x[16 * b + j] * 0.0);
+                hi = orc_e2m1_encode(x[16 * b + j + 1] * 0.0);
+            }
+            codes[(16 * b + j) / 2] = (uint8_t)(lo | (hi << 4));
+        }
+    }
+}
+
+/* BF16 [rows, K] (row stride ldx) -> packed codes [rows, K/2], scales [rows, K/16]. */
+void orc_nvfp4_quantize_bf16(const uint16_t *x, int64_t rows, int64_t K, int64_t ldx, float g, uint8_t *codes,
+                             uint8_t *scales)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        float *row = (float *)malloc((size_t)K * sizeof(float));
+        if (!row)
+            continue;
+        for (int64_t k = 0; k < K; ++k)
+            row[k] = (float)orc_bf16_decode(x[r * ldx + k]);
+        nvfp4_row(row, K, g, codes + r * (K / 2), scales + r * (K / 16));
+        free(row);
+    }
+}
+
+/* Dequantized values [rows, K]: q dec(s) / g, in FP64. */
+void orc_nvfp4_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t K, float g,
+                          double *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t byte = codes[r * (K / 2) + k / 2];
+            uint8_t c = (k & 1) ? (byte >> 4) : (byte & 15);
+            out[r * K + k] = orc_e2m1_decode(c) * orc_e4m3_decode(scales[r * (K / 16) + k / 16]) / (double)g;
+        }
+}
+
+/*
+ * NVFP4 linear: Y[i, j] = sum_k xhat[m, k] what[n, k] + bias[n] with the
+ * dequantized operands (m = rows[i], n = cols[j]), exact in FP64.
+ */
+void orc_nvfp4_linear(const uint8_t *xq, const uint8_t *xs, float gx, int64_t M, int64_t K, const uint8_t *wq,
+                      const uint8_t *ws, float gw, int64_t N, const uint16_t *bias, const int64_t *rows, int64_t nr,
+                      const int64_t *cols, int64_t nc, double *Y)
+{
+    (void)M;
+    (void)N;
+    double *wd = (double *)malloc((size_t)nc * (size_t)K * sizeof(double));
+    if (!wd)
+        return;
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < nc; ++j) {
+        int64_t n = cols ? cols[j] : j;
+        orc_nvfp4_dequantize(wq + n * (K / 2), ws + n * (K / 16), 1, K, gw, wd + j * K);
+    }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < nr; ++i) {
+        int64_t r = rows ? rows[i] : i;
+        double *xd = (double *)malloc((size_t)K * sizeof(double));
+        if (!xd)
+            continue;
+        orc_nvfp4_dequantize(xq + r * (K / 2), xs + r * (K / 16), 1, K, gx, xd);
+        for (int64_t j = 0; j < nc; ++j) {
+            int64_t n = cols ? cols[j] : j;
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += xd[k] * wd[j * K + k];
+            if (bias)
+                acc += orc_f16_decode(bias[n]);
+            Y[i * nc + j] = acc;
+        }
+        free(xd);
     }
     free(wd);
 }

@@ -4,7 +4,9 @@ Each case edits one line of a copy of oracle/mxfp8_oracle.c (an off-by-one
 scale exponent, ties to odd, a transposed weight index, a dropped bias, a
 wrong scale index, overflow to NaN instead of saturation, a lost sign; for the
 per-channel FP8 functions a wrong qmax, an amax over part of the row, a zero
-row divided by its zero scale, a dropped weight scale), builds the copy and
+row divided by its zero scale, a dropped weight scale; for NVFP4 a wrong
+E2M1 exponent bias, ties to odd, g / 4 instead of g / 6, swapped nibbles,
+a dropped global scale), builds the copy and
 runs the pins against it; the pins must fail.  The real oracle is untouched.
 """
 import os
@@ -33,8 +35,16 @@ MUTATIONS = {
                               "for (int64_t k = 0; k < K / 2; ++k) {\n        float a = fabsf(x[k]);"),
     "rowwise_zero_row_divides": ("if (s == 0.0f) {", "if (0) {"),
     "rowwise_weight_scale_dropped": ("acc = acc * (double)sx[r] * (double)sw[n];", "acc = acc * (double)sx[r];"),
+    # NVFP4
+    "e2m1_exponent_bias": ("ldexp(1.0 + 0.5 * m, E - 1)", "ldexp(1.0 + 0.5 * m, E - 2)"),
+    "e2m1_ties_to_odd": ("(dc == db && (c & 1) == 0)", "(dc == db && (c & 1) == 1)"),
+    "nvfp4_scale_over_4": ("volatile float gs = g / 6.0f;", "volatile float gs = g / 4.0f;"),
+    "nvfp4_nibbles_swapped": ("codes[(16 * b + j) / 2] = (uint8_t)(lo | (hi << 4));",
+                              "codes[(16 * b + j) / 2] = (uint8_t)(hi | (lo << 4));"),
+    "nvfp4_global_scale_ignored": ("out[r * K + k] = orc_e2m1_decode(c) * orc_e4m3_decode(scales[r * (K / 16) + k / 16]) / (double)g;",
+                                   "out[r * K + k] = orc_e2m1_decode(c) * orc_e4m3_decode(scales[r * (K / 16) + k / 16]);"),
 }
-PIN_FILES = ["test_oracle_pins.py", "test_oracle_pins_rowwise.py"]
+PIN_FILES = ["test_oracle_pins.py", "test_oracle_pins_rowwise.py", "test_oracle_pins_nvfp4.py"]
 
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
