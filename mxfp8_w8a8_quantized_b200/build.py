@@ -16,8 +16,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmxfp8.so")
 
-PUBLIC_HEADERS = ["mxfp8.h", "fp8_rowwise.h"]
-SOURCES = ["mxfp8_quant.cu", "mxfp8_gemm.cu", "mxfp8_capi.cu", "mxfp8_noalloc.cu", "fp8_rowwise.cu"]
+PUBLIC_HEADERS = ["mxfp8.h", "fp8_rowwise.h", "nvfp4.h"]
+SOURCES = ["mxfp8_quant.cu", "mxfp8_gemm.cu", "mxfp8_capi.cu", "mxfp8_noalloc.cu", "fp8_rowwise.cu", "nvfp4.cu"]
 HEADERS = ["ptx.cuh", "mx_element.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -7,6 +7,7 @@
 
 #include "fp8_rowwise.h"
 #include "mxfp8.h"
+#include "nvfp4.h"
 
 namespace mx {
 cudaError_t launch_quantize(const void *X, bool f32_in, int64_t M, int64_t K, int64_t ldx, uint8_t *Q, uint8_t *S,
@@ -15,6 +16,9 @@ cudaError_t launch_gelu(const void *X, void *Y, int64_t n, cudaStream_t stream);
 int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void *Wq, const void *Ws, int64_t N,
                 const void *bias, void *Y, int epi, void *S, cudaStream_t stream, unsigned long long timeout_ns,
                 cudaError_t *err);
+cudaError_t launch_nvfp4_quantize(const void *X, bool f32_in, int64_t M, int64_t K, int64_t ldx, float g,
+                                  uint8_t *Q, uint8_t *S, cudaStream_t stream);
+cudaError_t launch_nvfp4_amax(const void *X, bool f32_in, int64_t n, unsigned int *out, cudaStream_t stream);
 cudaError_t read_and_clear_status(unsigned int *out);
 cudaError_t launch_fp8_rowwise_quantize(const void *X, bool f32_in, int64_t M, int64_t K, int64_t ldx, uint8_t *Q,
                                         float *S, cudaStream_t stream, unsigned long long timeout_ns);
@@ -299,6 +303,69 @@ mxfp8_status fp8rw_linear(const void *X, int64_t M, int64_t K, const void *Wq, c
     if (st != MXFP8_OK)
         return st;
     return fp8rw_gemm(codes, scales, M, K, Wq, Wscale, N, bias, Y, stream);
+}
+
+/* --------------------------------------------------------------- NVFP4 */
+
+size_t nvfp4_scale_bytes(int64_t rows, int64_t K)
+{
+    if (rows < 0 || K <= 0 || K % 16 != 0)
+        return 0;
+    return (size_t)((rows + 127) / 128) * (size_t)((K + 63) / 64) * 512u;
+}
+
+static mxfp8_status nvfp4_amax_any(const void *X, bool f32, int64_t n, float *amax, mxfp8_stream_t stream)
+{
+    if (n < 0 || !amax)
+        return MXFP8_ERR_ARG;
+    if (n > 0 && !X)
+        return MXFP8_ERR_ARG;
+    if (n % 16 != 0)
+        return MXFP8_ERR_SHAPE;
+    if (!aligned(X, 16) || !aligned(amax, 4))
+        return MXFP8_ERR_ALIGN;
+    return from_cuda(mx::launch_nvfp4_amax(X, f32, n, reinterpret_cast<unsigned int *>(amax),
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mxfp8_status nvfp4_amax_bf16(const void *X, int64_t n, float *amax, mxfp8_stream_t stream)
+{
+    return nvfp4_amax_any(X, false, n, amax, stream);
+}
+
+mxfp8_status nvfp4_amax_f32(const float *W, int64_t n, float *amax, mxfp8_stream_t stream)
+{
+    return nvfp4_amax_any(W, true, n, amax, stream);
+}
+
+static mxfp8_status nvfp4_quantize_any(const void *X, bool f32, int64_t M, int64_t K, int64_t ldx, float g,
+                                       void *codes, void *scales, mxfp8_stream_t stream)
+{
+    if (M < 0 || K <= 0 || ldx < K || !(g > 0.0f) || !(g < 3.0e38f))
+        return MXFP8_ERR_ARG;
+    if (M == 0)
+        return MXFP8_OK;
+    if (!X || !codes || !scales)
+        return MXFP8_ERR_ARG;
+    if (K % 16 != 0 || M > kMaxRows || K > kMaxK)
+        return MXFP8_ERR_SHAPE;
+    if (!aligned(X, 16) || (ldx * (f32 ? 4 : 2)) % 16 != 0 || !aligned(codes, 8) || !aligned(scales, 4))
+        return MXFP8_ERR_ALIGN;
+    return from_cuda(mx::launch_nvfp4_quantize(X, f32, M, K, ldx, g, static_cast<uint8_t *>(codes),
+                                               static_cast<uint8_t *>(scales),
+                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mxfp8_status nvfp4_quantize_bf16(const void *X, int64_t M, int64_t K, int64_t ldx, float global_scale, void *codes,
+                                 void *scales, mxfp8_stream_t stream)
+{
+    return nvfp4_quantize_any(X, false, M, K, ldx, global_scale, codes, scales, stream);
+}
+
+mxfp8_status nvfp4_quantize_weight_f32(const float *W, int64_t N, int64_t K, float global_scale, void *Wq,
+                                       void *Wscale, mxfp8_stream_t stream)
+{
+    return nvfp4_quantize_any(W, true, N, K, K, global_scale, Wq, Wscale, stream);
 }
 
 mxfp8_status mxfp8_device_status(mxfp8_stream_t stream)

@@ -1,0 +1,239 @@
+/*
+ * nvfp4.cu -- NVFP4 quantization (sm_100a): packed E2M1 codes with one UE4M3
+ * scale per 16 elements and an FP32 global scale per tensor (page "Wan2.2
+ * I2V A14B, four-step 720p: native LightX2V FP8 and NVFP4", "Conversion and
+ * compatibility": packed E2M1 weights with E4M3 block scales, FP32
+ * input_global_scale and alpha fields; weights enter the quantizer as BF16).
+ *
+ * Per 16-element block, all in binary32 (the readings the oracle states):
+ *   s = UE4M3(RN(amax * RN(g / 6)))       nearest even, saturating at 448
+ *   q = E2M1(RN(x * RN(g / dec(s))))      nearest even, saturating at 6
+ * A block whose scale is 0 gets codes +-0.  Codes are packed two per byte,
+ * the even element in the low nibble; scales go straight into the
+ * tensor-core layout (512-byte atoms of 128 rows x 4 blocks, now 64 K
+ * elements per atom).
+ *
+ * HBM-bound: 2 (BF16) or 4 (FP32) bytes read, 0.5 + 1/16 byte written per
+ * element.  One lane owns one block (16 elements, two 16-byte loads), so the
+ * block amax needs no shuffle; a warp covers 512 elements of a row; four
+ * lanes' scale bytes form one 32-bit word of an atom.  Two segments are in
+ * flight per warp and the row / segment walk has no division in the loop.
+ * FP32 weights are rounded to BF16 (nearest even) on load.
+ */
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace mx {
+
+constexpr int NQ_THREADS = 256;
+constexpr int NQ_UNROLL = 2;
+
+/* 16 elements of a row as 8 words of BF16 pairs. */
+template <bool F32_IN>
+__device__ __forceinline__ void nq_load16(uint32_t (&w)[8], const void *base, int64_t elem_off)
+{
+    if constexpr (F32_IN) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const float *>(base) + elem_off);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint4 v = __ldcs(p + i);
+            __nv_bfloat162 a = __floats2bfloat162_rn(__uint_as_float(v.x), __uint_as_float(v.y));
+            __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(v.z), __uint_as_float(v.w));
+            w[2 * i] = *reinterpret_cast<uint32_t *>(&a);
+            w[2 * i + 1] = *reinterpret_cast<uint32_t *>(&b);
+        }
+    } else {
+        const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(base) + elem_off);
+        const uint4 a = __ldcs(p), b = __ldcs(p + 1);
+        w[0] = a.x, w[1] = a.y, w[2] = a.z, w[3] = a.w, w[4] = b.x, w[5] = b.y, w[6] = b.z, w[7] = b.w;
+    }
+}
+
+/* 8 values -> 4 bytes of E2M1 pairs (even element in the low nibble). */
+__device__ __forceinline__ uint32_t nq_e2m1x8(float x0, float x1, float x2, float x3, float x4, float x5, float x6,
+                                              float x7)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}\n"
+        : "=r"(r)
+        : "f"(x0), "f"(x1), "f"(x2), "f"(x3), "f"(x4), "f"(x5), "f"(x6), "f"(x7));
+    return r;
+}
+
+/*
+ * X [M, K] (row stride ldx) -> Q [M, K/2] packed codes, S scales (tensor-core
+ * layout, kg = ceil(K / 64) atoms per 128 rows).  Work unit = (row r,
+ * segment j of 512 elements); lane l owns block 32 j + l.  Rows in [M, Mrows)
+ * only write zero scale padding.
+ */
+template <bool F32_IN>
+__global__ void __launch_bounds__(NQ_THREADS) nvfp4_quantize_kernel(const void *__restrict__ X, int64_t M, int64_t K,
+                                                                    int64_t ldx, float g, uint8_t *__restrict__ Q,
+                                                                    uint8_t *__restrict__ S, int64_t Mrows,
+                                                                    int64_t nseg, int64_t kg)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warp0 = ((int64_t)blockIdx.x * NQ_THREADS + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * NQ_THREADS) >> 5;
+    const int64_t units = Mrows * nseg;
+    const int nblocks = (int)(K >> 4);
+    const float gs = __fdiv_rn(g, 6.0f);
+    const int64_t stride = nwarps * NQ_UNROLL;
+    const int nseg32 = (int)nseg;
+    const int stride_r = (int)(stride / nseg), stride_j = (int)(stride - (int64_t)stride_r * nseg);
+    int64_t u0 = warp0 * NQ_UNROLL;
+    int r0 = (int)(u0 / nseg), j0 = (int)(u0 - (int64_t)r0 * nseg);
+    const int M32 = (int)M, K32 = (int)K;
+
+    for (; u0 < units; u0 += stride) {
+        uint32_t w[NQ_UNROLL][8];
+        int row[NQ_UNROLL], k0[NQ_UNROLL];
+        bool valid[NQ_UNROLL];
+        {
+            int r = r0, j = j0;
+#pragma unroll
+            for (int i = 0; i < NQ_UNROLL; ++i) {
+                row[i] = r;
+                k0[i] = j * 512 + lane * 16;
+                valid[i] = (u0 + i < units) && (r < M32) && (k0[i] < K32);
+                if (valid[i])
+                    nq_load16<F32_IN>(w[i], X, (int64_t)r * ldx + k0[i]);
+                if (++j == nseg32) {
+                    j = 0;
+                    ++r;
+                }
+            }
+        }
+        r0 += stride_r;
+        j0 += stride_j;
+        if (j0 >= nseg32) {
+            j0 -= nseg32;
+            ++r0;
+        }
+#pragma unroll
+        for (int i = 0; i < NQ_UNROLL; ++i) {
+            if (u0 + i >= units) /* warp-uniform */
+                break;
+            uint32_t sb = 0u;
+            if (valid[i]) {
+                /* non-negative BF16 bit patterns order like their values */
+                uint32_t m2 = 0u;
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    m2 = __vmaxu2(m2, w[i][k] & 0x7FFF7FFFu);
+                const float amax = __uint_as_float(max(m2 << 16, m2 & 0xFFFF0000u));
+                sb = (uint32_t)__nv_cvt_float_to_fp8(amax * gs, __NV_SATFINITE, __NV_E4M3) & 0x7Fu;
+                const __half_raw hr = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)sb, __NV_E4M3);
+                const float ds = __half2float(__half(hr));
+                const float mul = ds > 0.0f ? __fdiv_rn(g, ds) : 0.0f;
+                float f[16];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    f[2 * k] = __uint_as_float(w[i][k] << 16) * mul;
+                    f[2 * k + 1] = __uint_as_float(w[i][k] & 0xFFFF0000u) * mul;
+                }
+                const uint32_t lo = nq_e2m1x8(f[0], f[1], f[2], f[3], f[4], f[5], f[6], f[7]);
+                const uint32_t hi = nq_e2m1x8(f[8], f[9], f[10], f[11], f[12], f[13], f[14], f[15]);
+                *reinterpret_cast<uint2 *>(Q + (int64_t)row[i] * (K >> 1) + (k0[i] >> 1)) = make_uint2(lo, hi);
+            }
+            /* word g (lanes 4g .. 4g+3) = blocks 32 j + 4g .. 32 j + 4g + 3 */
+            const uint32_t word = sb | (__shfl_down_sync(0xFFFFFFFFu, sb, 1) << 8) |
+                                  (__shfl_down_sync(0xFFFFFFFFu, sb, 2) << 16) |
+                                  (__shfl_down_sync(0xFFFFFFFFu, sb, 3) << 24);
+            if ((lane & 3) == 0) {
+                const int r = row[i];
+                const int b = (k0[i] >> 4); /* this lane's block = first block of the word */
+                if (b < nblocks) {
+                    const int64_t off = ((((int64_t)(r >> 7)) * kg + (b >> 2)) << 9) + ((r & 31) << 4) +
+                                        (((r >> 5) & 3) << 2);
+                    *reinterpret_cast<uint32_t *>(S + off) = word;
+                }
+            }
+        }
+    }
+}
+
+/* Largest magnitude of a tensor (after rounding FP32 input to BF16), as the
+ * bit pattern of a binary32, max-combined into *out. */
+template <bool F32_IN>
+__global__ void __launch_bounds__(256) nvfp4_amax_kernel(const void *__restrict__ X, int64_t n16,
+                                                         unsigned int *__restrict__ out)
+{
+    uint32_t m2 = 0u;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += (int64_t)gridDim.x * blockDim.x) {
+        uint32_t w[8];
+        nq_load16<F32_IN>(w, X, i * 16);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            m2 = __vmaxu2(m2, w[k] & 0x7FFF7FFFu);
+    }
+    uint32_t m = max(m2 << 16, m2 & 0xFFFF0000u);
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    if ((threadIdx.x & 31) == 0 && m != 0u)
+        atomicMax(out, m);
+}
+
+static int nq_num_sms()
+{
+    static int sms[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return 148;
+    if (sms[dev] == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+            v = 148;
+        sms[dev] = v;
+    }
+    return sms[dev];
+}
+
+cudaError_t launch_nvfp4_quantize(const void *X, bool f32_in, int64_t M, int64_t K, int64_t ldx, float g,
+                                  uint8_t *Q, uint8_t *S, cudaStream_t stream)
+{
+    const int64_t Mrows = ((M + 127) / 128) * 128;
+    const int64_t nseg = (K + 511) / 512;
+    const int64_t kg = (K / 16 + 3) / 4;
+    const int64_t units = Mrows * nseg;
+    if (units == 0)
+        return cudaSuccess;
+    const int64_t per_block = (NQ_THREADS / 32) * NQ_UNROLL;
+    int64_t blocks = (units + per_block - 1) / per_block;
+    const int64_t cap = (int64_t)nq_num_sms() * 8 * 4; /* 8 resident blocks x 4 waves */
+    if (blocks > cap)
+        blocks = cap;
+    if (f32_in)
+        nvfp4_quantize_kernel<true><<<(unsigned)blocks, NQ_THREADS, 0, stream>>>(X, M, K, ldx, g, Q, S, Mrows, nseg, kg);
+    else
+        nvfp4_quantize_kernel<false><<<(unsigned)blocks, NQ_THREADS, 0, stream>>>(X, M, K, ldx, g, Q, S, Mrows, nseg,
+                                                                                  kg);
+    return cudaGetLastError();
+}
+
+/* n % 16 == 0; *out (device) receives the amax bits (cleared first). */
+cudaError_t launch_nvfp4_amax(const void *X, bool f32_in, int64_t n, unsigned int *out, cudaStream_t stream)
+{
+    cudaError_t e = cudaMemsetAsync(out, 0, sizeof(unsigned int), stream);
+    if (e != cudaSuccess || n == 0)
+        return e;
+    const int64_t n16 = n / 16;
+    int64_t blocks = (n16 + 255) / 256;
+    const int64_t cap = (int64_t)nq_num_sms() * 8;
+    if (blocks > cap)
+        blocks = cap;
+    if (f32_in)
+        nvfp4_amax_kernel<true><<<(unsigned)blocks, 256, 0, stream>>>(X, n16, out);
+    else
+        nvfp4_amax_kernel<false><<<(unsigned)blocks, 256, 0, stream>>>(X, n16, out);
+    return cudaGetLastError();
+}
+
+} // namespace mx

@@ -54,6 +54,17 @@ _lib.fp8rw_linear_workspace_bytes.argtypes = [_I64, _I64]
 _lib.fp8rw_linear_workspace_bytes.restype = _SZ
 _lib.fp8rw_linear.argtypes = [_P, _I64, _I64, _P, _P, _I64, _P, _P, _P, _SZ, _P]
 _lib.fp8rw_linear.restype = ctypes.c_int
+_F = ctypes.c_float
+_lib.nvfp4_scale_bytes.argtypes = [_I64, _I64]
+_lib.nvfp4_scale_bytes.restype = _SZ
+_lib.nvfp4_amax_bf16.argtypes = [_P, _I64, _P, _P]
+_lib.nvfp4_amax_bf16.restype = ctypes.c_int
+_lib.nvfp4_amax_f32.argtypes = [_P, _I64, _P, _P]
+_lib.nvfp4_amax_f32.restype = ctypes.c_int
+_lib.nvfp4_quantize_bf16.argtypes = [_P, _I64, _I64, _I64, _F, _P, _P, _P]
+_lib.nvfp4_quantize_bf16.restype = ctypes.c_int
+_lib.nvfp4_quantize_weight_f32.argtypes = [_P, _I64, _I64, _F, _P, _P, _P]
+_lib.nvfp4_quantize_weight_f32.restype = ctypes.c_int
 _lib.mxfp8_device_status.argtypes = [_P]
 _lib.mxfp8_device_status.restype = ctypes.c_int
 
@@ -67,7 +78,9 @@ EXPORTS = ("mxfp8_status_str", "mxfp8_scale_bytes", "mxfp8_quantize", "mxfp8_qua
            "mxfp8_gelu_tanh_bf16", "mxfp8_device_status", "mxfp8_linear_noalloc",
            "mxfp8_gemm_quantize_out",
            "fp8rw_quantize_bf16", "fp8rw_quantize_weight_f32", "fp8rw_gemm", "fp8rw_linear_workspace_bytes",
-           "fp8rw_linear")
+           "fp8rw_linear",
+           "nvfp4_scale_bytes", "nvfp4_amax_bf16", "nvfp4_amax_f32", "nvfp4_quantize_bf16",
+           "nvfp4_quantize_weight_f32")
 
 
 class MXFP8Error(RuntimeError):
@@ -260,6 +273,57 @@ def fp8rw_linear(x: torch.Tensor, wq, wscale, bias=None, out=None, workspace=Non
     _check(_lib.fp8rw_linear(_ptr(x), M, K, _ptr(wq), _ptr(wscale), N, _ptr(bias), _ptr(out), _ptr(workspace),
                              workspace.numel(), _stream()), "fp8rw_linear")
     return out
+
+
+# ---------------------------------------------------------------- NVFP4
+def nvfp4_scale_bytes(rows: int, K: int) -> int:
+    return int(_lib.nvfp4_scale_bytes(rows, K))
+
+
+def nvfp4_amax(t: torch.Tensor) -> torch.Tensor:
+    """amax of a contiguous BF16 or FP32 tensor (FP32 measured after
+    rounding to BF16), as a 1-element FP32 CUDA tensor."""
+    if not t.is_cuda or not t.is_contiguous() or t.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("t must be a contiguous BF16 or FP32 CUDA tensor")
+    out = torch.empty(1, dtype=torch.float32, device=t.device)
+    f = _lib.nvfp4_amax_bf16 if t.dtype == torch.bfloat16 else _lib.nvfp4_amax_f32
+    _check(f(_ptr(t), t.numel(), _ptr(out), _stream()), "nvfp4_amax")
+    return out
+
+
+def nvfp4_global_scale(amax: float) -> float:
+    """448 * 6 / amax in binary32 (the tensor's largest block gets the
+    largest UE4M3 scale)."""
+    import numpy as np
+    return float(np.float32(np.float32(448.0 * 6.0) / np.float32(amax)))
+
+
+def nvfp4_quantize(x: torch.Tensor, global_scale: float, codes=None, scales=None):
+    """BF16 [M, K] -> (packed E2M1 codes uint8 [M, K/2], UE4M3 scales, tensor-core layout)."""
+    if not x.is_cuda or x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D BF16 CUDA tensor")
+    M, K = x.shape
+    ldx = x.stride(0) if M > 1 else K
+    if x.stride(1) != 1 or ldx < K:
+        raise ValueError("x must have unit column stride and row stride >= K")
+    if codes is None:
+        codes = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(max(nvfp4_scale_bytes(M, K), 1), dtype=torch.uint8, device=x.device)
+    _check(_lib.nvfp4_quantize_bf16(_ptr(x), M, K, ldx, global_scale, _ptr(codes), _ptr(scales), _stream()),
+           "nvfp4_quantize_bf16")
+    return codes, scales
+
+
+def nvfp4_quantize_weight(w: torch.Tensor, global_scale: float):
+    """FP32 [N, K] (rounded to BF16 first) -> (packed codes [N, K/2], scales)."""
+    _cuda(w, "w", torch.float32)
+    N, K = w.shape
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device)
+    scales = torch.empty(max(nvfp4_scale_bytes(N, K), 1), dtype=torch.uint8, device=w.device)
+    _check(_lib.nvfp4_quantize_weight_f32(_ptr(w), N, K, global_scale, _ptr(codes), _ptr(scales), _stream()),
+           "nvfp4_quantize_weight_f32")
+    return codes, scales
 
 
 def device_status() -> int:

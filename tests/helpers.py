@@ -17,11 +17,12 @@ def bf16_values(bits: np.ndarray) -> np.ndarray:
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
 
 
-def tc_index(rows: int, K: int):
-    """For every (r, b) of a [rows, K/32] scale matrix, its byte offset in the
-    tensor-core layout: 512-byte atoms of 128 rows x 4 blocks, atom (i, j) at
-    (i * ceil(K/128) + j) * 512, byte (r, b) inside at (r%32)*16 + (r//32 % 4)*4 + b%4."""
-    nb = K // 32
+def tc_index(rows: int, K: int, block: int = 32):
+    """For every (r, b) of a [rows, K/block] scale matrix, its byte offset in
+    the tensor-core layout: 512-byte atoms of 128 rows x 4 blocks, atom (i, j)
+    at (i * ceil(K/(4 block)) + j) * 512, byte (r, b) inside at
+    (r%32)*16 + (r//32 % 4)*4 + b%4."""
+    nb = K // block
     kg = (nb + 3) // 4
     r = np.arange(rows)[:, None]
     b = np.arange(nb)[None, :]
@@ -32,8 +33,8 @@ def tc_bytes(rows: int, K: int) -> int:
     return ((rows + 127) // 128) * ((K + 127) // 128) * 512
 
 
-def unswizzle(sc: np.ndarray, rows: int, K: int) -> np.ndarray:
-    return sc[tc_index(rows, K)]
+def unswizzle(sc: np.ndarray, rows: int, K: int, block: int = 32) -> np.ndarray:
+    return sc[tc_index(rows, K, block)]
 
 
 def tol_violations(y: np.ndarray, yref: np.ndarray):

@@ -9,7 +9,7 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 INCLUDE = os.path.join(ROOT, "include")
-PREFIXES = ("mxfp8_", "fp8rw_")
+PREFIXES = ("mxfp8_", "fp8rw_", "nvfp4_")
 
 
 def declared_functions():
