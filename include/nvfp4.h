@@ -12,9 +12,13 @@
  *                                       even, saturating at 448
  *     q = E2M1(RN(x * RN(g / dec(s))))  nearest even, saturating at 6;
  *                                       s = 0 gives q = +-0
- *   dequantized value q * dec(s) / g (the layer computes
- *     Y[m, n] = BF16_RNE(alpha * sum_k qx sx qw sw + F32(bias[n]))
- *   with alpha = 1 / (g_x * g_w); this library provides the quantizers).
+ *   dequantized value q * dec(s) / g; the layer computes
+ *     Y[m, n] = BF16_RNE(alpha * sum_k (qx dec(sx)) (qw dec(sw)) + F32(bias[n]))
+ *   with alpha = 1 / (g_x * g_w) and FP32 accumulation.  Each product
+ *   q * dec(s) is exact in FP16 (at most 6 significant bits), so the GEMM
+ *   expands the codes to FP16 in the SM and runs on the FP16 tensor-core
+ *   kind; the sum is that of a block-scaled 4-bit MMA up to the order of
+ *   the FP32 additions.
  *
  * A convenient global scale is g = 448 * 6 / amax(tensor) (nvfp4_amax_*),
  * which gives the tensor's largest block the largest scale.  For
@@ -59,6 +63,33 @@ mxfp8_status nvfp4_quantize_bf16(const void *X, int64_t M, int64_t K, int64_t ld
 /* Weights: FP32 W [N, K] rounded to BF16 (nearest even), then as above. */
 mxfp8_status nvfp4_quantize_weight_f32(const float *W, int64_t N, int64_t K, float global_scale, void *Wq,
                                        void *Wscale, mxfp8_stream_t stream);
+
+/*
+ * The GEMM and epilogue on quantized operands: Xq [M, K/2] and Wq [N, K/2]
+ * packed codes with their scales (nvfp4_scale_bytes of [M, K] and [N, K]),
+ * alpha = 1 / (g_x g_w) (finite, > 0), bias F16 [N] or NULL, Y BF16 [M, N]
+ * (written).  Requires K % 64 == 0, N % 8 == 0, N > 0, M >= 0, every pointer
+ * 16-byte aligned.
+ */
+mxfp8_status nvfp4_gemm(const void *Xq, const void *Xscale, int64_t M, int64_t K, const void *Wq,
+                        const void *Wscale, int64_t N, float alpha, const void *bias, void *Y,
+                        mxfp8_stream_t stream);
+
+/* Workspace bytes nvfp4_linear needs: the activation codes (rounded up to
+ * 256 bytes) and their scales. */
+size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t K);
+
+/*
+ * The whole layer: nvfp4_quantize_bf16 of X (row stride K) with the
+ * activation global scale x_global_scale into `workspace`, then nvfp4_gemm
+ * with alpha = 1 / (x_global_scale * w_global_scale) (w_global_scale: the
+ * scale the weights were quantized with).  workspace: >=
+ * nvfp4_linear_workspace_bytes(M, K) bytes, 256-byte aligned, overwritten.
+ * Requirements as nvfp4_gemm.
+ */
+mxfp8_status nvfp4_linear(const void *X, int64_t M, int64_t K, float x_global_scale, const void *Wq,
+                          const void *Wscale, int64_t N, float w_global_scale, const void *bias, void *Y,
+                          void *workspace, size_t ws_bytes, mxfp8_stream_t stream);
 
 #ifdef __cplusplus
 }

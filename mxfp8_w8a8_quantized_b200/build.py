@@ -17,8 +17,15 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmxfp8.so")
 
 PUBLIC_HEADERS = ["mxfp8.h", "fp8_rowwise.h", "nvfp4.h"]
-SOURCES = ["mxfp8_quant.cu", "mxfp8_gemm.cu", "mxfp8_capi.cu", "mxfp8_noalloc.cu", "fp8_rowwise.cu", "nvfp4.cu"]
-HEADERS = ["ptx.cuh", "mx_element.cuh"]
+SOURCES = ["mxfp8_quant.cu", "mxfp8_gemm.cu", "mxfp8_capi.cu", "mxfp8_noalloc.cu", "fp8_rowwise.cu", "nvfp4.cu",
+           "nvfp4_gemm.cu"]
+HEADERS = ["ptx.cuh", "mx_element.cuh", "tmap_host.cuh"]
+# The files each profiled kernel is compiled from: a profile summary names
+# the hash of its kernel's files, so that it goes stale only when they change.
+KERNEL_FILES = {
+    "mxfp8_gemm": ["mxfp8_gemm.cu", "ptx.cuh", "mx_element.cuh", "tmap_host.cuh"],
+    "nvfp4_gemm": ["nvfp4_gemm.cu", "ptx.cuh", "tmap_host.cuh"],
+}
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -35,10 +42,16 @@ def _inputs():
             + [os.path.join(INCLUDE, h) for h in PUBLIC_HEADERS] + [os.path.abspath(__file__)])
 
 
-def source_sha() -> str:
-    """Hash of the kernel sources; ties a profile summary to one build."""
+def source_sha(kernel: str = None) -> str:
+    """Hash of the library's sources, or of one kernel's files
+    (KERNEL_FILES); ties a profile summary to one build."""
+    if kernel is None:
+        paths = ([os.path.join(CSRC, s) for s in SOURCES + HEADERS]
+                 + [os.path.join(INCLUDE, h) for h in PUBLIC_HEADERS])
+    else:
+        paths = [os.path.join(CSRC, s) for s in KERNEL_FILES[kernel]]
     h = hashlib.sha256()
-    for p in [os.path.join(CSRC, s) for s in SOURCES + HEADERS] + [os.path.join(INCLUDE, h) for h in PUBLIC_HEADERS]:
+    for p in paths:
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

@@ -23,6 +23,10 @@ cudaError_t read_and_clear_status(unsigned int *out);
 cudaError_t launch_fp8_rowwise_quantize(const void *X, bool f32_in, int64_t M, int64_t K, int64_t ldx, uint8_t *Q,
                                         float *S, cudaStream_t stream, unsigned long long timeout_ns);
 cudaError_t read_and_clear_rw_status(unsigned int *out);
+int launch_nvfp4_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void *Wq, const void *Ws,
+                      int64_t N, float alpha, const void *bias, void *Y, cudaStream_t stream,
+                      unsigned long long timeout_ns, cudaError_t *err);
+cudaError_t read_and_clear_nv_status(unsigned int *out);
 } // namespace mx
 
 namespace {
@@ -368,15 +372,74 @@ mxfp8_status nvfp4_quantize_weight_f32(const float *W, int64_t N, int64_t K, flo
     return nvfp4_quantize_any(W, true, N, K, K, global_scale, Wq, Wscale, stream);
 }
 
+mxfp8_status nvfp4_gemm(const void *Xq, const void *Xscale, int64_t M, int64_t K, const void *Wq,
+                        const void *Wscale, int64_t N, float alpha, const void *bias, void *Y,
+                        mxfp8_stream_t stream)
+{
+    if (M < 0 || K <= 0 || N <= 0 || !(alpha > 0.0f) || !(alpha < 3.0e38f))
+        return MXFP8_ERR_ARG;
+    if (M == 0)
+        return MXFP8_OK;
+    if (!Xq || !Xscale || !Wq || !Wscale || !Y)
+        return MXFP8_ERR_ARG;
+    if (K % 64 != 0 || N % 8 != 0 || M > kMaxRows || N > kMaxRows || K > kMaxK)
+        return MXFP8_ERR_SHAPE;
+    if (!aligned(Xq, 16) || !aligned(Xscale, 16) || !aligned(Wq, 16) || !aligned(Wscale, 16) || !aligned(Y, 16) ||
+        (bias && !aligned(bias, 16)))
+        return MXFP8_ERR_ALIGN;
+    cudaError_t e;
+    int r = mx::launch_nvfp4_gemm(Xq, Xscale, M, K, Wq, Wscale, N, alpha, bias, Y,
+                                  reinterpret_cast<cudaStream_t>(stream), kWaitLimitNs, &e);
+    if (r == 1)
+        return MXFP8_ERR_CUDA;
+    return r == 0 ? MXFP8_OK : from_cuda(e);
+}
+
+size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t K)
+{
+    if (M < 0 || K <= 0 || K % 16 != 0)
+        return 0;
+    return round_up((size_t)M * (size_t)(K / 2), 256) + nvfp4_scale_bytes(M, K);
+}
+
+mxfp8_status nvfp4_linear(const void *X, int64_t M, int64_t K, float x_global_scale, const void *Wq,
+                          const void *Wscale, int64_t N, float w_global_scale, const void *bias, void *Y,
+                          void *workspace, size_t ws_bytes, mxfp8_stream_t stream)
+{
+    if (M < 0 || K <= 0 || N <= 0 || !(x_global_scale > 0.0f) || !(w_global_scale > 0.0f) ||
+        !(x_global_scale < 3.0e38f) || !(w_global_scale < 3.0e38f))
+        return MXFP8_ERR_ARG;
+    if (M == 0)
+        return MXFP8_OK;
+    if (!X || !workspace)
+        return MXFP8_ERR_ARG;
+    if (K % 64 != 0)
+        return MXFP8_ERR_SHAPE;
+    if (!aligned(workspace, 256) || !aligned(X, 16))
+        return MXFP8_ERR_ALIGN;
+    if (ws_bytes < nvfp4_linear_workspace_bytes(M, K))
+        return MXFP8_ERR_ARG;
+    const double a = 1.0 / ((double)x_global_scale * (double)w_global_scale);
+    if (!(a > 0.0) || !(a < 3.0e38))
+        return MXFP8_ERR_ARG;
+    uint8_t *codes = static_cast<uint8_t *>(workspace);
+    uint8_t *scales = codes + round_up((size_t)M * (size_t)(K / 2), 256);
+    mxfp8_status st = nvfp4_quantize_bf16(X, M, K, K, x_global_scale, codes, scales, stream);
+    if (st != MXFP8_OK)
+        return st;
+    return nvfp4_gemm(codes, scales, M, K, Wq, Wscale, N, (float)a, bias, Y, stream);
+}
+
 mxfp8_status mxfp8_device_status(mxfp8_stream_t stream)
 {
     cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess)
         return MXFP8_ERR_CUDA;
-    unsigned int word = 0, rw_word = 0;
-    if (mx::read_and_clear_status(&word) != cudaSuccess || mx::read_and_clear_rw_status(&rw_word) != cudaSuccess)
+    unsigned int word = 0, rw_word = 0, nv_word = 0;
+    if (mx::read_and_clear_status(&word) != cudaSuccess || mx::read_and_clear_rw_status(&rw_word) != cudaSuccess ||
+        mx::read_and_clear_nv_status(&nv_word) != cudaSuccess)
         return MXFP8_ERR_CUDA;
-    return (word | rw_word) ? MXFP8_ERR_TIMEOUT : MXFP8_OK;
+    return (word | rw_word | nv_word) ? MXFP8_ERR_TIMEOUT : MXFP8_OK;
 }
 
 } // extern "C"

@@ -62,6 +62,7 @@
 
 #include "mx_element.cuh"
 #include "ptx.cuh"
+#include "tmap_host.cuh"
 
 namespace mx {
 
@@ -703,37 +704,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 }
 
 /* ------------------------------------------------------------ host side */
-typedef CUresult (*PFN_encodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                    const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static PFN_encodeTiled get_encode_fn()
-{
-    static PFN_encodeTiled fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_encodeTiled>(p);
-    }
-    return fn;
-}
-
 /* K-major E4M3 operand [rows, K]: box 128 (K bytes) x box_rows, 128-byte swizzle. */
 static bool make_operand_map(CUtensorMap *m, const void *base, int64_t rows, int64_t K, uint32_t box_rows)
 {
-    PFN_encodeTiled enc = get_encode_fn();
-    if (!enc)
-        return false;
-    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)K};
-    cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, K, rows, K, (uint32_t)BK, box_rows,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 /* Scale array in the tensor-core layout viewed as [row blocks][K/128][128 u32]
@@ -758,32 +733,14 @@ static bool make_scale_map(CUtensorMap *m, const void *base, int64_t rows, int64
  * epilogue's staging layout); stores are clipped at M and N. */
 static bool make_output_map(CUtensorMap *m, void *base, int64_t M, int64_t N)
 {
-    PFN_encodeTiled enc = get_encode_fn();
-    if (!enc)
-        return false;
-    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
-    cuuint64_t strides[1] = {(cuuint64_t)(N * 2)};
-    cuuint32_t box[2] = {32, 32};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 /* MXFP8 codes out [M, N] (quantizing epilogues): box 64 bytes x 32 rows,
  * 64-byte swizzle (same staging layout as the BF16 boxes); clipped at M. */
 static bool make_codes_out_map(CUtensorMap *m, void *base, int64_t M, int64_t N)
 {
-    PFN_encodeTiled enc = get_encode_fn();
-    if (!enc)
-        return false;
-    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
-    cuuint64_t strides[1] = {(cuuint64_t)N};
-    cuuint32_t box[2] = {64, 32};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, N, M, N, 64, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 struct DevInfo {

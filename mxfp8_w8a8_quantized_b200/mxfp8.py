@@ -65,6 +65,12 @@ _lib.nvfp4_quantize_bf16.argtypes = [_P, _I64, _I64, _I64, _F, _P, _P, _P]
 _lib.nvfp4_quantize_bf16.restype = ctypes.c_int
 _lib.nvfp4_quantize_weight_f32.argtypes = [_P, _I64, _I64, _F, _P, _P, _P]
 _lib.nvfp4_quantize_weight_f32.restype = ctypes.c_int
+_lib.nvfp4_gemm.argtypes = [_P, _P, _I64, _I64, _P, _P, _I64, _F, _P, _P, _P]
+_lib.nvfp4_gemm.restype = ctypes.c_int
+_lib.nvfp4_linear_workspace_bytes.argtypes = [_I64, _I64]
+_lib.nvfp4_linear_workspace_bytes.restype = _SZ
+_lib.nvfp4_linear.argtypes = [_P, _I64, _I64, _F, _P, _P, _I64, _F, _P, _P, _P, _SZ, _P]
+_lib.nvfp4_linear.restype = ctypes.c_int
 _lib.mxfp8_device_status.argtypes = [_P]
 _lib.mxfp8_device_status.restype = ctypes.c_int
 
@@ -80,7 +86,7 @@ EXPORTS = ("mxfp8_status_str", "mxfp8_scale_bytes", "mxfp8_quantize", "mxfp8_qua
            "fp8rw_quantize_bf16", "fp8rw_quantize_weight_f32", "fp8rw_gemm", "fp8rw_linear_workspace_bytes",
            "fp8rw_linear",
            "nvfp4_scale_bytes", "nvfp4_amax_bf16", "nvfp4_amax_f32", "nvfp4_quantize_bf16",
-           "nvfp4_quantize_weight_f32")
+           "nvfp4_quantize_weight_f32", "nvfp4_gemm", "nvfp4_linear_workspace_bytes", "nvfp4_linear")
 
 
 class MXFP8Error(RuntimeError):
@@ -322,8 +328,46 @@ def nvfp4_quantize_weight(w: torch.Tensor, global_scale: float):
     codes = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device)
     scales = torch.empty(max(nvfp4_scale_bytes(N, K), 1), dtype=torch.uint8, device=w.device)
     _check(_lib.nvfp4_quantize_weight_f32(_ptr(w), N, K, global_scale, _ptr(codes), _ptr(scales), _stream()),
-           "nvfp4_quantize_weight_f32")
+           "nvfp4_quantize_weight_f32", "nvfp4_gemm", "nvfp4_linear_workspace_bytes", "nvfp4_linear")
     return codes, scales
+
+
+def nvfp4_alpha(x_global_scale: float, w_global_scale: float) -> float:
+    """alpha = 1 / (g_x g_w), rounded once to binary32 (as nvfp4_linear)."""
+    import numpy as np
+    return float(np.float32(1.0 / (float(x_global_scale) * float(w_global_scale))))
+
+
+def nvfp4_gemm(xq, xscale, wq, wscale, alpha: float, bias=None, out=None):
+    """Y = BF16(alpha sum_k (qx dec(sx)) (qw dec(sw)) + bias) from NVFP4
+    operands: packed codes [M, K/2] / [N, K/2] and their scales."""
+    M, K2 = xq.shape
+    N = wq.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    _check(_lib.nvfp4_gemm(_ptr(xq), _ptr(xscale), M, 2 * K2, _ptr(wq), _ptr(wscale), N, alpha, _ptr(bias),
+                           _ptr(out), _stream()), "nvfp4_gemm")
+    return out
+
+
+def nvfp4_linear_workspace_bytes(M: int, K: int) -> int:
+    return int(_lib.nvfp4_linear_workspace_bytes(M, K))
+
+
+def nvfp4_linear(x: torch.Tensor, x_global_scale: float, wq, wscale, w_global_scale: float, bias=None, out=None,
+                 workspace=None):
+    """The NVFP4 layer: quantize x with its global scale, then nvfp4_gemm
+    with alpha = 1 / (g_x g_w)."""
+    _cuda(x, "x", torch.bfloat16)
+    M, K = x.shape
+    N = wq.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(max(nvfp4_linear_workspace_bytes(M, K), 256), dtype=torch.uint8, device=x.device)
+    _check(_lib.nvfp4_linear(_ptr(x), M, K, x_global_scale, _ptr(wq), _ptr(wscale), N, w_global_scale, _ptr(bias),
+                             _ptr(out), _ptr(workspace), workspace.numel(), _stream()), "nvfp4_linear")
+    return out
 
 
 def device_status() -> int:

@@ -148,6 +148,31 @@ def test_fp8_rowwise_argument_checks_return_before_launch(lib):
     assert L.fp8rw_linear(FAKE, 4, 128, FAKE, FAKE, 16, None, FAKE, FAKE + 16, need, None) == ALIGN
 
 
+def test_nvfp4_gemm_argument_checks_return_before_launch(lib):
+    P, I64, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float
+    lib.nvfp4_gemm.argtypes = [P, P, I64, I64, P, P, I64, F, P, P, P]
+    lib.nvfp4_linear_workspace_bytes.argtypes = [I64, I64]
+    lib.nvfp4_linear_workspace_bytes.restype = ctypes.c_size_t
+    lib.nvfp4_linear.argtypes = [P, I64, I64, F, P, P, I64, F, P, P, P, ctypes.c_size_t, P]
+    L = lib
+    ARG, ALIGN, SHAPE = 1, 2, 3
+    assert L.nvfp4_gemm(FAKE, FAKE, 4, 96, FAKE, FAKE, 16, 1.0, None, FAKE, None) == SHAPE    # K % 64
+    assert L.nvfp4_gemm(FAKE, FAKE, 4, 128, FAKE, FAKE, 12, 1.0, None, FAKE, None) == SHAPE   # N % 8
+    assert L.nvfp4_gemm(FAKE, FAKE + 4, 4, 128, FAKE, FAKE, 16, 1.0, None, FAKE, None) == ALIGN
+    assert L.nvfp4_gemm(FAKE, FAKE, 4, 128, FAKE, FAKE, 16, 1.0, FAKE + 2, FAKE, None) == ALIGN  # bias
+    assert L.nvfp4_gemm(FAKE, FAKE, 4, 128, FAKE, FAKE, 16, 0.0, None, FAKE, None) == ARG     # alpha > 0
+    assert L.nvfp4_gemm(FAKE, FAKE, 4, 128, FAKE, FAKE, 16, float("inf"), None, FAKE, None) == ARG
+    assert L.nvfp4_gemm(FAKE, FAKE, 4, 128, FAKE, None, 16, 1.0, None, FAKE, None) == ARG
+    assert L.nvfp4_gemm(FAKE, FAKE, 0, 128, FAKE, FAKE, 16, 1.0, None, FAKE, None) == 0
+    need = L.nvfp4_linear_workspace_bytes(4, 128)
+    assert need == 256 + 2 * 512                 # codes rounded to 256 B + one row block of 2 scale atoms
+    assert L.nvfp4_linear(FAKE, 4, 128, 1.0, FAKE, FAKE, 16, 1.0, None, FAKE, FAKE, need - 1, None) == ARG
+    assert L.nvfp4_linear(FAKE, 4, 128, 1.0, FAKE, FAKE, 16, 1.0, None, FAKE, FAKE + 16, need, None) == ALIGN
+    assert L.nvfp4_linear(FAKE, 4, 96, 1.0, FAKE, FAKE, 16, 1.0, None, FAKE, FAKE, need, None) == SHAPE
+    assert L.nvfp4_linear(FAKE, 4, 128, 0.0, FAKE, FAKE, 16, 1.0, None, FAKE, FAKE, need, None) == ARG
+    assert L.nvfp4_linear(FAKE, 4, 128, 1e-30, FAKE, FAKE, 16, 1e-30, None, FAKE, FAKE, need, None) == ARG
+
+
 def test_product_fails_loudly_without_library(tmp_path, monkeypatch):
     import importlib.util
     import sys

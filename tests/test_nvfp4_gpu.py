@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import bf16_bits, bf16_values, unswizzle
+from helpers import assert_within_tol, bf16_bits, bf16_values, unswizzle
 from mxfp8_w8a8_quantized_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -65,3 +65,98 @@ def test_weight_quantizer_rounds_to_bf16_first(mx, N, K):
     rq, rs = oracle.nvfp4_quantize_bf16(wb, g)
     assert np.array_equal(codes.cpu().numpy(), rq)
     assert np.array_equal(unswizzle(scales.cpu().numpy(), N, K, 16), rs)
+
+
+# ------------------------------------------------------------------ GEMM
+# Y within |Y - Yref| <= 2^-7 |Yref| + 1e-3 rms(Yref) of the exact (FP64)
+# oracle; the FP32 accumulation order is not fixed, alpha is rounded once to
+# binary32.
+
+def _nv_layer(mx, M, K, N, seed, with_bias=True):
+    x = synth.activations_device(M, K, seed, 0, "cuda")
+    w = synth.weights_device(N, K, seed, 0, "cuda")
+    b = synth.bias_device(N, seed, 0, "cuda") if with_bias else None
+    gx, _ = _g(mx, x)
+    gw, _ = _g(mx, w)
+    wq, ws = mx.nvfp4_quantize_weight(w, gw)
+    return x, w, b, gx, gw, wq, ws
+
+
+def _oracle_y(x, w, b, gx, gw, rows=None, cols=None):
+    rq, rs = oracle.nvfp4_quantize_bf16(bf16_bits(x), gx)
+    oq, os_ = oracle.nvfp4_quantize_bf16(bf16_bits(w.to(torch.bfloat16)), gw)
+    bb = None if b is None else b.cpu().view(torch.int16).numpy().view(np.uint16)
+    return oracle.nvfp4_linear(rq, rs, gx, oq, os_, gw, bb, rows=rows, cols=cols)
+
+
+@pytest.mark.parametrize("M,K,N", [(256, 512, 512), (300, 512, 384), (1, 64, 8), (129, 256, 640),
+                                   (1000, 1088, 1536), (517, 13824, 264), (260, 320, 520)])
+def test_gemm_within_tolerance(mx, M, K, N):
+    x, w, b, gx, gw, wq, ws = _nv_layer(mx, M, K, N, seed=M + N)
+    xq, xs = mx.nvfp4_quantize(x, gx)
+    y = mx.nvfp4_gemm(xq, xs, wq, ws, mx.nvfp4_alpha(gx, gw), b)
+    y2 = mx.nvfp4_linear(x, gx, wq, ws, gw, b)
+    torch.cuda.synchronize()
+    assert mx.device_status() == 0
+    assert torch.equal(y, y2), "nvfp4_linear differs from quantize + gemm"
+    yref = _oracle_y(x, w, b, gx, gw)
+    assert_within_tol(bf16_values(bf16_bits(y)), yref, f"nvfp4 {M}x{K}x{N}")
+
+
+def test_gemm_exact_grid_values(mx):
+    # every block holds a 6 and values of the E2M1 grid; with g = 1 every
+    # scale is exactly 1 (6 * RN(1/6) rounds to 1 in E4M3), the codes are
+    # the values themselves, and the FP32 sums are exact (multiples of 1/4
+    # below 2^20), so Y is the BF16 rounding of the exact result
+    M, K, N = 130, 256, 136
+    grid = torch.tensor([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    gen = torch.Generator(device="cpu").manual_seed(7)
+
+    def make(rows):
+        v = grid[torch.randint(0, 8, (rows, K), generator=gen)]
+        v = v * torch.where(torch.rand((rows, K), generator=gen) < 0.5, -1.0, 1.0)
+        v[:, ::16] = 6.0
+        return v
+
+    xv, wv = make(M), make(N)
+    x = xv.to(torch.bfloat16).cuda()
+    xq, xs = mx.nvfp4_quantize(x, 1.0)
+    wq, ws = mx.nvfp4_quantize_weight(wv.cuda(), 1.0)
+    y = mx.nvfp4_gemm(xq, xs, wq, ws, 1.0, None)
+    torch.cuda.synchronize()
+    assert np.all(unswizzle(xs.cpu().numpy(), M, K, 16) == 0x38)
+    exact = xv.double().numpy() @ wv.double().numpy().T
+    assert np.array_equal(bf16_bits(y), oracle.bf16_rne(exact))
+
+
+def test_gemm_q_projection_480p_full_size_sampled(mx):
+    """M = 32760, K = N = 5120: codes and scales bit-exact, sampled Y."""
+    M, K, N, seed = synth.TOKENS_480P, synth.HIDDEN, synth.HIDDEN, 1
+    x, w, b, gx, gw, wq, ws = _nv_layer(mx, M, K, N, seed)
+    xq, xs = mx.nvfp4_quantize(x, gx)
+    y = mx.nvfp4_gemm(xq, xs, wq, ws, mx.nvfp4_alpha(gx, gw), b)
+    torch.cuda.synchronize()
+    assert mx.device_status() == 0
+    rq, rs = oracle.nvfp4_quantize_bf16(bf16_bits(x), gx)
+    assert np.array_equal(xq.cpu().numpy(), rq)
+    assert np.array_equal(unswizzle(xs.cpu().numpy(), M, K, 16), rs)
+    oq, os_ = oracle.nvfp4_quantize_bf16(bf16_bits(w.to(torch.bfloat16)), gw)
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([[0, 127, 128, 255, 256, M - 129, M - 1], np.arange(M - 40, M),
+                                     rng.choice(M, 150, replace=False)]))
+    cols = np.unique(np.concatenate([[0, 8, 255, 256, N - 1], rng.choice(N, 120, replace=False)]))
+    bb = b.cpu().view(torch.int16).numpy().view(np.uint16)
+    yref = oracle.nvfp4_linear(rq, rs, gx, oq, os_, gw, bb, rows=rows, cols=cols)
+    got = y[torch.from_numpy(rows).cuda()][:, torch.from_numpy(cols).cuda()]
+    assert_within_tol(bf16_values(bf16_bits(got)), yref, "nvfp4 Q projection")
+
+
+def test_gemm_argument_errors(mx):
+    x = torch.zeros((4, 96), dtype=torch.bfloat16, device="cuda")
+    xq, xs = mx.nvfp4_quantize(x, 1.0)
+    w = torch.zeros((8, 96), dtype=torch.float32, device="cuda")
+    wq, ws = mx.nvfp4_quantize_weight(w, 1.0)
+    with pytest.raises(mx.MXFP8Error):          # K = 96 is not a multiple of 64
+        mx.nvfp4_gemm(xq, xs, wq, ws, 1.0)
+    with pytest.raises(mx.MXFP8Error):          # alpha must be finite and > 0
+        mx.nvfp4_gemm(xq, xs, wq, ws, 0.0)
