@@ -328,7 +328,7 @@ def nvfp4_quantize_weight(w: torch.Tensor, global_scale: float):
     codes = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device)
     scales = torch.empty(max(nvfp4_scale_bytes(N, K), 1), dtype=torch.uint8, device=w.device)
     _check(_lib.nvfp4_quantize_weight_f32(_ptr(w), N, K, global_scale, _ptr(codes), _ptr(scales), _stream()),
-           "nvfp4_quantize_weight_f32", "nvfp4_gemm", "nvfp4_linear_workspace_bytes", "nvfp4_linear")
+           "nvfp4_quantize_weight_f32")
     return codes, scales
 
 

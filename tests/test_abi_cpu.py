@@ -185,3 +185,18 @@ def test_product_fails_loudly_without_library(tmp_path, monkeypatch):
     with pytest.raises(ImportError):
         spec.loader.exec_module(mod)
     assert "mxfp8_copy" not in sys.modules
+
+
+def test_binding_checks_every_status_with_its_entry_name():
+    """Each C call in the binding goes through _check(status, name), the
+    name being the entry point called."""
+    import ast
+    src = open(os.path.join(ROOT, "mxfp8_w8a8_quantized_b200", "mxfp8.py")).read()
+    calls = [n for n in ast.walk(ast.parse(src)) if isinstance(n, ast.Call) and getattr(n.func, "id", None) == "_check"]
+    assert calls
+    for c in calls:
+        assert len(c.args) == 2, ast.unparse(c)[:120]
+        status, name = c.args
+        assert isinstance(status, ast.Call) and isinstance(name, ast.Constant)
+        if isinstance(status.func, ast.Attribute):      # _lib.<entry>(...); else a chosen entry
+            assert status.func.attr == name.value, ast.unparse(c)[:120]
