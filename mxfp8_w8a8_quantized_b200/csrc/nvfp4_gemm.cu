@@ -22,26 +22,28 @@
  *
  * Persistent kernel on CTA pairs (cluster of 2, tcgen05.mma.cta_group::2):
  * 256 x 256 output tiles, each CTA holding 128 rows of A and 128 rows of B.
- * Roles (320 threads per CTA):
- *   warp 0      TMA producer: per 256-wide K step ("raw stage") the CTA's
- *               128 x 128-byte boxes of A and B codes (128-byte swizzle) and
- *               the four 512-byte scale atoms of its A rows and B rows (one
- *               bulk copy each), into a 2-deep ring.
- *   warp 1      allocates 256 TMEM columns; in the leader CTA one thread
- *               issues, per 64-wide K step, four kind::f16 MMAs of K = 16
- *               and commits the step's release to both CTAs.
- *   warps 2..9  expand and write back.  Each thread owns one row (threads
- *               0..127 of A, 128..255 of B) and, per 64-wide K step, turns
- *               its 32 code bytes and 4 scale bytes into 64 FP16 values
- *               (cvt.rn.f16x2.e2m1x2, exact multiply by the scale) stored in
- *               the 128-byte-swizzled K-major layout the MMA reads, into a
- *               4-deep ring; the generic-proxy stores are fenced to the async
- *               proxy and announced to the leader's barrier (16 arrivals per
- *               step, both CTAs).  Between K steps, once the next tile's
- *               first ring slots are filled, the same warps drain the
- *               finished accumulator (one tcgen05.ld of 32 lanes x 128
- *               columns per warp), release it at once, and write Y through
- *               swizzled smem boxes and TMA stores.
+ * Roles (576 threads per CTA):
+ *   warp 0       TMA producer: per 128-wide K step ("code stage") the CTA's
+ *                128 x 64-byte boxes of A and B codes (64-byte swizzle) and
+ *                the two 512-byte scale atoms of its A rows and B rows (one
+ *                bulk copy each), into a 3-deep ring.
+ *   warp 1       allocates 512 TMEM columns (two 256-column accumulators);
+ *                in the leader CTA one thread issues, per 64-wide K step,
+ *                four kind::f16 MMAs of K = 16 into the tile's accumulator
+ *                and commits the step's release to both CTAs.
+ *   warps 2..17  expand and write back.  Two threads per row (A rows, then
+ *                B rows), each owning 32 elements of every 64-wide K step:
+ *                per code stage a thread turns 2 x 16 code bytes and 2 x 2
+ *                scale bytes into 64 FP16 values (cvt.rn.f16x2.e2m1x2, exact
+ *                multiply by the scale) stored in the 128-byte-swizzled
+ *                K-major layout the MMA reads, into a 4-deep ring; the
+ *                generic-proxy stores are fenced to the async proxy and
+ *                announced to the leader's barriers (32 arrivals per step,
+ *                both CTAs).  Once the next tile's first ring slots are
+ *                filled, the same warps drain the previous tile's
+ *                accumulator in 32-column pieces (the MMA meanwhile runs the
+ *                next tile into the other accumulator) and write Y through
+ *                swizzled smem boxes and TMA stores.
  * Every wait is bounded: on timeout the kernel records the timeout in a
  * device status word, drains its own MMAs, frees TMEM and returns.
  */
@@ -58,34 +60,37 @@ namespace nv {
 
 using namespace mx;
 
-constexpr int XW = 8;                    /* expand / epilogue warps */
+constexpr int XW = 16;                   /* expand / epilogue warps */
 constexpr int THREADS = (2 + XW) * 32;
 constexpr int FS = 4;                    /* FP16 operand stages */
-constexpr int RS = 2;                    /* code / scale stages */
+constexpr int RS = 3;                    /* code / scale stages */
 constexpr int KF = 64;                   /* K elements per FP16 stage (128-byte rows) */
-constexpr int KR = 256;                  /* K elements per code stage (128 bytes of codes per row) */
+constexpr int KR = 128;                  /* K elements per code stage (64 bytes of codes per row) */
 constexpr int SUB = KR / KF;             /* FP16 stages per code stage */
 constexpr int TILE_M = 256, TILE_N = 256;
-constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t TILE_BYTES = 128 * 128; /* 128 rows x 128 bytes */
-constexpr uint32_t SF_BYTES = SUB * 512;   /* four 64-wide scale atoms of 128 rows */
+constexpr uint32_t TMEM_COLS = 512;      /* two 256-column FP32 accumulators */
+constexpr uint32_t TILE_BYTES = 128 * 128; /* FP16 operand slot: 128 rows x 128 bytes */
+constexpr uint32_t CODE_BYTES = 128 * 64;  /* code slot: 128 rows x 64 bytes */
+constexpr uint32_t SF_BYTES = SUB * 512;   /* two 64-wide scale atoms of 128 rows */
 constexpr uint32_t OFF_FA = 0;
 constexpr uint32_t OFF_FB = OFF_FA + FS * TILE_BYTES;
 constexpr uint32_t OFF_RA = OFF_FB + FS * TILE_BYTES;
-constexpr uint32_t OFF_RB = OFF_RA + RS * TILE_BYTES;
-constexpr uint32_t OFF_SA = OFF_RB + RS * TILE_BYTES;
+constexpr uint32_t OFF_RB = OFF_RA + RS * CODE_BYTES;
+constexpr uint32_t OFF_SA = OFF_RB + RS * CODE_BYTES;
 constexpr uint32_t OFF_SB = OFF_SA + RS * SF_BYTES;
 constexpr uint32_t OFF_EPI = OFF_SB + RS * SF_BYTES;
 constexpr uint32_t EPI_BUF = 32 * 32 * 2; /* 32 rows x 32 BF16 */
 constexpr uint32_t OFF_BAR = OFF_EPI + XW * EPI_BUF;
-/* full[FS], empty[FS], rfull[RS], rempty[RS], tfull, tempty, drain */
-constexpr uint32_t NUM_BARS = 2 * FS + 2 * RS + 3;
+/* full[FS], empty[FS], rfull[RS], rempty[RS], tfull[2], tempty[2], drain */
+constexpr uint32_t NUM_BARS = 2 * FS + 2 * RS + 5;
 constexpr uint32_t OFF_TMEMPTR = OFF_BAR + NUM_BARS * 8;
 constexpr uint32_t OFF_ABORT = OFF_TMEMPTR + 4;
 constexpr uint32_t SMEM_USED = OFF_TMEMPTR + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024; /* slack to align the base to 1 KiB */
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(OFF_EPI % 1024 == 0 && OFF_RA % 1024 == 0, "swizzled buffers must be 1 KiB aligned");
+static_assert(SUB == 2 && FS % 2 == 0, "a pass expands the two K steps of one code stage into a ring-slot pair");
+static_assert(OFF_RA % 1024 == 0 && OFF_RB % 1024 == 0 && OFF_EPI % 1024 == 0 && CODE_BYTES % 1024 == 0,
+              "swizzled buffers must be 1 KiB aligned");
 constexpr int RASTER_SMALL_B = 8, RASTER_LARGE_B = 16;
 constexpr int64_t RASTER_LARGE_B_BYTES = 48ll << 20; /* weight bytes above which 16 M tiles share a group */
 constexpr uint32_t SUSPEND_NS = 1000000u;
@@ -119,24 +124,6 @@ __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t a)
     uint32_t v;
     asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
     return v;
-}
-/* Wait with acquire at cluster scope: the phase was completed by arrivals
- * (release, cluster scope) of threads in both CTAs of the pair. */
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity, uint32_t suspend_ns)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(suspend_ns)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t cluster_addr)
-{
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 /* D (+)= A . B^T over the CTA pair, FP16 x FP16 -> FP32, K = 16 per MMA. */
 __device__ __forceinline__ void tc_mma_f16_pair(uint32_t tacc, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -177,17 +164,6 @@ __device__ __forceinline__ void expand_word(uint32_t w, uint32_t s2, uint32_t &h
         : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
         : "r"(w), "r"(s2));
 }
-/* UE4M3 scale byte -> the FP16 pair (dec(s), dec(s)) */
-__device__ __forceinline__ uint32_t scale_pair(uint32_t sbyte)
-{
-    uint32_t d;
-    asm("{\n\t.reg .b16 t;\n\t"
-        "cvt.u16.u32 t, %1;\n\t"
-        "cvt.rn.f16x2.e4m3x2 %0, t;\n\t}\n"
-        : "=r"(d)
-        : "r"(sbyte * 0x101u));
-    return d;
-}
 
 /* Tile t -> (M tile, N tile): `raster` M tiles are walked together for
  * every N tile so that their A rows stay in L2 while the weights stream. */
@@ -207,18 +183,14 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int ras
  * timeout it records ST_TIMEOUT in the device status word and raises the
  * CTA's abort flag, so the other roles stop waiting too.
  */
-template <bool CLUSTER>
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, unsigned long long limit_ns,
                                              volatile uint32_t *abort_flag)
 {
-    auto probe = [&]() {
-        return CLUSTER ? mbar_try_wait_cluster(bar, parity, SUSPEND_NS) : mbar_try_wait(bar, parity, SUSPEND_NS);
-    };
-    if (probe())
+    if (mbar_try_wait(bar, parity, SUSPEND_NS))
         return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        if (probe())
+        if (mbar_try_wait(bar, parity, SUSPEND_NS))
             return true;
         if (*abort_flag)
             return false;
@@ -233,80 +205,114 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, unsi
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, unsigned long long limit_ns,
                                           volatile uint32_t *abort_flag)
 {
-    const bool ok = wait_bounded<false>(bar, parity, limit_ns, abort_flag);
+    const bool ok = wait_bounded(bar, parity, limit_ns, abort_flag);
     return __all_sync(0xFFFFFFFFu, ok);
 }
 
-/*
- * One thread, one row, one 64-wide K step: 32 code bytes (two 16-byte
- * chunks of the row's 128-byte swizzled code line) and the row's 4 scale
- * bytes of the step's atom -> 64 FP16 values, written as 8 chunks of the
- * 128-byte swizzled FP16 row.
- */
-__device__ __forceinline__ void expand_row_step(uint32_t code_row, uint32_t sf_word_addr, bool have_scales, int j,
-                                                uint32_t f16_row, uint32_t x)
+/* scale bytes (b, b, c, c) of a word -> FP16 pairs (dec(b), dec(b)) and
+ * (dec(c), dec(c)) */
+__device__ __forceinline__ void scale_pairs2(uint32_t d, uint32_t &lo, uint32_t &hi)
 {
-    const uint4 c0 = ld_shared_v4(code_row + ((((uint32_t)(2 * j)) ^ x) << 4));
-    const uint4 c1 = ld_shared_v4(code_row + ((((uint32_t)(2 * j + 1)) ^ x) << 4));
-    const uint32_t sw = have_scales ? ld_shared_u32(sf_word_addr) : 0u;
-    const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+    asm("{\n\t.reg .b16 l, h;\n\t"
+        "mov.b32 {l, h}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, l;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}\n"
+        : "=r"(lo), "=r"(hi)
+        : "r"(d));
+}
+
+/*
+ * One thread, half a row (32 elements), the NS (1 or 2) 64-wide K steps of
+ * one code stage.  Step j reads the 16-byte code chunk 2 j + h of the row's
+ * 64-byte code line (64-byte swizzle: chunk ^ ((row / 2) % 4)) and the
+ * scale bytes 2h, 2h + 1 of the row's word in atom j, and writes 32 FP16
+ * values as chunks 4h .. 4h + 3 of the row in step j's operand slot
+ * (128-byte swizzle: chunk ^ (row % 8)).  All loads are issued first.
+ */
+template <int NS>
+__device__ __forceinline__ void expand_half_row(uint32_t code_row, uint32_t xc, uint32_t sf_word_addr,
+                                                bool have_scales, int h, uint32_t f16_row0, uint32_t f16_row1,
+                                                uint32_t xf)
+{
+    uint4 c[NS];
+    uint32_t sw[NS];
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-        const uint32_t s2 = scale_pair((sw >> (8 * b)) & 0xFFu);
+    for (int j = 0; j < NS; ++j)
+        c[j] = ld_shared_v4(code_row + ((((uint32_t)(2 * j + h)) ^ xc) << 4));
 #pragma unroll
-        for (int hch = 0; hch < 2; ++hch) {
-            const int c = 2 * b + hch; /* FP16 chunk = 8 elements = one code word */
+    for (int j = 0; j < NS; ++j)
+        sw[j] = have_scales ? ld_shared_u32(sf_word_addr + (uint32_t)j * 512u) : 0u;
+#pragma unroll
+    for (int j = 0; j < NS; ++j) {
+        uint32_t s_lo, s_hi;
+        scale_pairs2(__byte_perm(sw[j], 0u, h ? 0x3322u : 0x1100u), s_lo, s_hi);
+        const uint32_t f16_row = j == 0 ? f16_row0 : f16_row1;
+        const uint32_t w[4] = {c[j].x, c[j].y, c[j].z, c[j].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { /* 8 elements; block i / 2 of the half */
             uint32_t h0, h1, h2, h3;
-            expand_word(w[c], s2, h0, h1, h2, h3);
-            st_shared_v4(f16_row + ((((uint32_t)c) ^ x) << 4), h0, h1, h2, h3);
+            expand_word(w[i], i < 2 ? s_lo : s_hi, h0, h1, h2, h3);
+            st_shared_v4(f16_row + ((((uint32_t)(4 * h + i)) ^ xf) << 4), h0, h1, h2, h3);
         }
     }
 }
 
-/* Y = BF16(alpha acc + bias), 32 columns at a time, staged through a
- * 64-byte-swizzled smem box and written by one TMA store per warp. */
-__device__ __forceinline__ void epilogue_store(const uint32_t (&acc)[128], const Params &p, const CUtensorMap *tmap_y,
-                                               int row0, int col0, int lane, uint32_t buf, uint32_t rowbase,
+/* 32 lanes x 32 consecutive 32-bit TMEM columns -> 32 registers, with the
+ * wait for the load in the same statement. */
+__device__ __forceinline__ void tmem_ld_32x32b_x32_sync(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+/* Y = BF16(alpha acc + bias) for 32 rows x 32 columns, staged through a
+ * 64-byte-swizzled smem box and written by one TMA store of the warp. */
+__device__ __forceinline__ void epilogue_piece(const uint32_t (&acc)[32], const Params &p, const CUtensorMap *tmap_y,
+                                               int row0, int colc, int lane, uint32_t buf, uint32_t rowbase,
                                                uint32_t swz)
 {
+    if (row0 >= p.M || colc >= p.N) /* whole box outside Y */
+        return;
+    if (lane == 0)
+        bulk_wait_group_read0(); /* previous box has left the buffer */
+    __syncwarp();
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        const int colc = col0 + 32 * c;
-        if (row0 >= p.M || colc >= p.N)
-            continue;
-        if (lane == 0)
-            bulk_wait_group_read0(); /* previous box has left the buffer */
-        __syncwarp();
-#pragma unroll
-        for (int j8 = 0; j8 < 4; ++j8) {
-            const int col = colc + 8 * j8;
-            float b[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            if (p.bias && col < p.N) {
-                const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(p.bias + col));
-                const __half2 *bh = reinterpret_cast<const __half2 *>(&bv);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float2 f2 = __half22float2(bh[j]);
-                    b[2 * j] = f2.x;
-                    b[2 * j + 1] = f2.y;
-                }
-            }
-            uint32_t o[4];
+    for (int j8 = 0; j8 < 4; ++j8) {
+        const int col = colc + 8 * j8;
+        float b[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (p.bias && col < p.N) {
+            const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(p.bias + col));
+            const __half2 *bh = reinterpret_cast<const __half2 *>(&bv);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const int a = 32 * c + 8 * j8 + 2 * j;
-                __nv_bfloat162 v = __floats2bfloat162_rn(fmaf(p.alpha, __uint_as_float(acc[a]), b[2 * j]),
-                                                         fmaf(p.alpha, __uint_as_float(acc[a + 1]), b[2 * j + 1]));
-                o[j] = *reinterpret_cast<uint32_t *>(&v);
+                const float2 f2 = __half22float2(bh[j]);
+                b[2 * j] = f2.x;
+                b[2 * j + 1] = f2.y;
             }
-            st_shared_v4(rowbase + ((((uint32_t)j8) ^ swz) << 4), o[0], o[1], o[2], o[3]);
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-            tma_store_2d(tmap_y, colc, row0, buf);
-            bulk_commit_group();
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int a = 8 * j8 + 2 * j;
+            __nv_bfloat162 v = __floats2bfloat162_rn(fmaf(p.alpha, __uint_as_float(acc[a]), b[2 * j]),
+                                                     fmaf(p.alpha, __uint_as_float(acc[a + 1]), b[2 * j + 1]));
+            o[j] = *reinterpret_cast<uint32_t *>(&v);
         }
+        st_shared_v4(rowbase + ((((uint32_t)j8) ^ swz) << 4), o[0], o[1], o[2], o[3]);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(tmap_y, colc, row0, buf);
+        bulk_commit_group();
     }
 }
 
@@ -329,9 +335,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t bar_empty = bar_full + FS * 8;     /* + 8 s */
     const uint32_t bar_rfull = bar_empty + FS * 8;    /* + 8 r, r < RS */
     const uint32_t bar_rempty = bar_rfull + RS * 8;   /* + 8 r */
-    const uint32_t bar_tfull = bar_rempty + RS * 8;
-    const uint32_t bar_tempty = bar_tfull + 8;
-    const uint32_t bar_drain = bar_tempty + 8;
+    const uint32_t bar_tfull = bar_rempty + RS * 8;   /* + 8 b, b < 2 */
+    const uint32_t bar_tempty = bar_tfull + 2 * 8;    /* + 8 b */
+    const uint32_t bar_drain = bar_tempty + 2 * 8;
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + OFF_TMEMPTR);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + OFF_ABORT);
 
@@ -345,8 +351,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(bar_rfull + 8 * r, 1);
             mbar_init(bar_rempty + 8 * r, XW);
         }
-        mbar_init(bar_tfull, 1);
-        mbar_init(bar_tempty, 2 * XW);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_tfull + 8 * b, 1);
+            mbar_init(bar_tempty + 8 * b, 2 * XW);
+        }
         mbar_init(bar_drain, 1);
         fence_mbar_init();
     }
@@ -380,16 +388,16 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const bool a_in = rowA < p.M, b_in = rowB < p.N; /* scale atoms exist for the row block */
                 for (int kr = 0; kr < KRN; ++kr, ++ir) {
                     const uint32_t s = ir % RS, ph = (ir / RS) & 1u;
-                    if (!wait_bounded<false>(bar_rempty + 8 * s, ph ^ 1u, lim, abort_flag)) {
+                    if (!wait_bounded(bar_rempty + 8 * s, ph ^ 1u, lim, abort_flag)) {
                         ok = false;
                         break;
                     }
                     const int n_at = min(SUB, p.kg - SUB * kr);
                     const uint32_t sf_bytes = (uint32_t)n_at * 512u;
                     const uint32_t full = bar_rfull + 8 * s;
-                    mbar_arrive_expect_tx(full, 2u * TILE_BYTES + (a_in ? sf_bytes : 0u) + (b_in ? sf_bytes : 0u));
-                    tma_load_2d(sbase + OFF_RA + s * TILE_BYTES, &tmap_a, kr * 128, rowA, full);
-                    tma_load_2d(sbase + OFF_RB + s * TILE_BYTES, &tmap_b, kr * 128, rowB, full);
+                    mbar_arrive_expect_tx(full, 2u * CODE_BYTES + (a_in ? sf_bytes : 0u) + (b_in ? sf_bytes : 0u));
+                    tma_load_2d(sbase + OFF_RA + s * CODE_BYTES, &tmap_a, kr * (KR / 2), rowA, full);
+                    tma_load_2d(sbase + OFF_RB + s * CODE_BYTES, &tmap_b, kr * (KR / 2), rowB, full);
                     if (a_in)
                         bulk_load(sbase + OFF_SA + s * SF_BYTES,
                                   p.sfa + ((size_t)(rowA / 128) * p.kg + (size_t)(SUB * kr)) * 512u, sf_bytes, full);
@@ -406,14 +414,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint32_t it = 0, tl = 0;
             bool ok = true, any = false;
             for (int t = tile0; ok && t < num_tiles; t += tstep, ++tl) {
-                if (!wait_bounded<true>(bar_tempty, (tl & 1u) ^ 1u, lim, abort_flag)) {
+                const uint32_t ab = tl & 1u; /* accumulator of this tile */
+                if (!wait_bounded(bar_tempty + 8 * ab, ((tl >> 1) & 1u) ^ 1u, lim, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                const uint32_t tacc = tmem + 256u * ab;
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const uint32_t s = it % FS, ph = (it / FS) & 1u;
-                    if (!wait_bounded<true>(bar_full + 8 * s, ph, lim, abort_flag)) {
+                    if (!wait_bounded(bar_full + 8 * s, ph, lim, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -422,41 +432,43 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const uint64_t bdesc = desc_kmajor_sw128(sbase + OFF_FB + s * TILE_BYTES);
 #pragma unroll
                     for (int k = 0; k < KF / 16; ++k)
-                        tc_mma_f16_pair(tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc,
+                        tc_mma_f16_pair(tacc, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc,
                                         (kb | k) != 0);
                     tc_commit_pair(bar_empty + 8 * s, (uint16_t)0x3);
                     any = true;
                 }
                 if (!ok)
                     break;
-                tc_commit_pair(bar_tfull, (uint16_t)0x3);
+                tc_commit_pair(bar_tfull + 8 * ab, (uint16_t)0x3);
             }
-            if (ok && tl > 0) {
+            if (ok) {
                 /* every epilogue (the peer's included) has released the last
-                 * accumulator, so no remote arrival is still in flight */
-                (void)wait_bounded<true>(bar_tempty, (tl & 1u) ^ 1u, lim, abort_flag);
+                 * accumulators, so no remote arrival is still in flight */
+                for (uint32_t u = tl > 2u ? tl - 2u : 0u; u < tl; ++u)
+                    (void)wait_bounded(bar_tempty + 8 * (u & 1u), (u >> 1) & 1u, lim, abort_flag);
             }
             if (!ok && any) {
                 /* wait for this thread's MMAs before TMEM is freed */
                 volatile uint32_t own = 0u;
                 tc_commit_pair(bar_drain, (uint16_t)0x1);
-                (void)wait_bounded<false>(bar_drain, 0u, lim, &own);
+                (void)wait_bounded(bar_drain, 0u, lim, &own);
             }
         }
     } else {
         /* ------------------------------------- expand + epilogue warps */
         const int e = (warp - 2) * 32 + lane;
-        const int op = e >> 7; /* 0: A row, 1: B row */
+        const int op = e >> 8;        /* 0: A row, 1: B row */
+        const int h = (e >> 7) & 1;   /* which 32 elements of each 64-wide K step */
         const int r = e & 127;
-        const uint32_t x = (uint32_t)(r & 7);
+        const uint32_t xc = (uint32_t)((r >> 1) & 3); /* 64-byte swizzle of the code line */
+        const uint32_t xf = (uint32_t)(r & 7);        /* 128-byte swizzle of the FP16 row */
         const uint32_t sf_off = (uint32_t)((r & 31) * 16 + ((r >> 5) & 3) * 4);
-        const uint32_t code_base = sbase + (op ? OFF_RB : OFF_RA) + (uint32_t)r * 128u;
+        const uint32_t code_base = sbase + (op ? OFF_RB : OFF_RA) + (uint32_t)r * 64u;
         const uint32_t sf_base = sbase + (op ? OFF_SB : OFF_SA) + sf_off;
         const uint32_t f16_base = sbase + (op ? OFF_FB : OFF_FA) + (uint32_t)r * 128u;
-        const uint32_t tempty_lead = mapa_shared(bar_tempty, 0u);
-        /* epilogue geometry: TMEM sub-partition and column half of this warp */
+        /* epilogue geometry: TMEM sub-partition and 64-column group */
         const int q = warp & 3;
-        const int h = (warp - 2) >> 2;
+        const int cg = (warp - 2) >> 2;
         const uint32_t buf = sbase + OFF_EPI + (uint32_t)(warp - 2) * EPI_BUF;
         const uint32_t rowbase = buf + (uint32_t)lane * 64u;
         const uint32_t swz = ((uint32_t)lane >> 1) & 3u;
@@ -465,24 +477,32 @@ __global__ void __launch_bounds__(THREADS, 1)
         bool ok = true;
         bool pending = false;
         int pend_t = 0;
-        /* drains the accumulator of tile pend_t and writes its Y */
+        /* drains the accumulator of tile pend_t in two 32-column pieces and
+         * writes its Y; the accumulator is released after the second load */
         auto epilogue = [&]() -> bool {
             int mb, nb;
             tile_coords(pend_t, p.num_m, p.num_n, p.raster, mb, nb);
-            const bool got = wait_bounded<false>(bar_tfull, tl & 1u, lim, abort_flag);
+            const uint32_t ab = tl & 1u;
+            const bool got = wait_bounded(bar_tfull + 8 * ab, (tl >> 1) & 1u, lim, abort_flag);
             if (!__all_sync(0xFFFFFFFFu, got))
                 return false;
             tc_fence_after();
-            uint32_t acc[128];
-            tmem_ld_32x32b_x128_sync(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(h * 128), acc);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive_cluster(tempty_lead);
-            ++tl;
             const int row0 = mb * TILE_M + (int)(rank * 128u) + 32 * q;
-            const int col0 = nb * TILE_N + h * 128;
-            epilogue_store(acc, p, &tmap_y, row0, col0, lane, buf, rowbase, swz);
+            const int col0 = nb * TILE_N + cg * 64;
+#pragma unroll 1
+            for (int c = 0; c < 2; ++c) {
+                uint32_t acc[32];
+                tmem_ld_32x32b_x32_sync(tmem + ((uint32_t)(32 * q) << 16) + 256u * ab + (uint32_t)(cg * 64 + 32 * c),
+                                        acc);
+                if (c == 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive_cluster(mapa_shared(bar_tempty + 8 * ab, 0u));
+                }
+                epilogue_piece(acc, p, &tmap_y, row0, col0 + 32 * c, lane, buf, rowbase, swz);
+            }
+            ++tl;
             return true;
         };
 
@@ -491,7 +511,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             tile_coords(t, p.num_m, p.num_n, p.raster, mb, nb);
             const int row_block = op ? nb * TILE_N + (int)(rank * 128u) : mb * TILE_M + (int)(rank * 128u);
             const bool have_scales = row_block < (op ? p.N : p.M);
-            for (int kb = 0; kb < KB; ++kb, ++it) {
+            /* one pass per code stage: its two K steps (one at an odd end) */
+            for (int kb = 0; kb < KB;) {
                 if (pending && kb == FS) {
                     pending = false;
                     if (!epilogue()) {
@@ -499,28 +520,39 @@ __global__ void __launch_bounds__(THREADS, 1)
                         break;
                     }
                 }
-                const int j = kb % SUB;
+                const int ns = kb + 1 < KB ? 2 : 1;
                 const uint32_t rs = ir % RS;
-                if (j == 0 && !warp_wait(bar_rfull + 8 * rs, (ir / RS) & 1u, lim, abort_flag)) {
+                const uint32_t s0 = it % FS, s1 = (it + 1) % FS;
+                if (!warp_wait(bar_rfull + 8 * rs, (ir / RS) & 1u, lim, abort_flag) ||
+                    !warp_wait(bar_empty + 8 * s0, ((it / FS) & 1u) ^ 1u, lim, abort_flag) ||
+                    (ns == 2 && !warp_wait(bar_empty + 8 * s1, (((it + 1) / FS) & 1u) ^ 1u, lim, abort_flag))) {
                     ok = false;
                     break;
                 }
-                const uint32_t s = it % FS;
-                if (!warp_wait(bar_empty + 8 * s, ((it / FS) & 1u) ^ 1u, lim, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                expand_row_step(code_base + rs * TILE_BYTES, sf_base + rs * SF_BYTES + (uint32_t)j * 512u,
-                                have_scales, j, f16_base + s * TILE_BYTES, x);
+                const uint32_t code_row = code_base + rs * CODE_BYTES;
+                const uint32_t sf_addr = sf_base + rs * SF_BYTES;
+                if (ns == 2)
+                    expand_half_row<2>(code_row, xc, sf_addr, have_scales, h, f16_base + s0 * TILE_BYTES,
+                                       f16_base + s1 * TILE_BYTES, xf);
+                else
+                    expand_half_row<1>(code_row, xc, sf_addr, have_scales, h, f16_base + s0 * TILE_BYTES, 0u, xf);
                 fence_proxy_async_smem(); /* generic-proxy stores -> visible to the tensor core */
                 __syncwarp();
-                if (lane == 0)
-                    mbar_arrive_release_cluster(mapa_shared(bar_full + 8 * s, 0u));
-                if (j == SUB - 1 || kb == KB - 1) {
-                    if (lane == 0)
-                        mbar_arrive(bar_rempty + 8 * rs);
-                    ++ir;
+                if (lane == 0) {
+                    /* every thread fenced its stores to the async proxy; one
+                     * arrive per warp on the leader's barrier (the peer's
+                     * through its shared::cluster address), as the
+                     * transform-to-MMA hand-off of the 2-SM UMMA pipelines
+                     * does.  A cluster-scope release here costs about 1,400
+                     * cycles per arrive and throttled the pair (measured). */
+                    mbar_arrive_cluster(mapa_shared(bar_full + 8 * s0, 0u));
+                    if (ns == 2)
+                        mbar_arrive_cluster(mapa_shared(bar_full + 8 * s1, 0u));
+                    mbar_arrive(bar_rempty + 8 * rs);
                 }
+                ++ir;
+                kb += ns;
+                it += (uint32_t)ns;
             }
             if (!ok)
                 break;
@@ -627,8 +659,8 @@ int launch_nvfp4_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, cons
         return 2;
     }
     CUtensorMap ma, mb, my;
-    if (!encode_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, K / 2, M, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K / 2, N, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+    if (!encode_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, K / 2, M, K / 2, nv::KR / 2, 128, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !encode_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K / 2, N, K / 2, nv::KR / 2, 128, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !encode_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
         return 1;
     nv::Params p;
