@@ -94,6 +94,10 @@ static_assert(OFF_RA % 1024 == 0 && OFF_RB % 1024 == 0 && OFF_EPI % 1024 == 0 &&
 constexpr int RASTER_SMALL_B = 8, RASTER_LARGE_B = 16;
 constexpr int64_t RASTER_LARGE_B_BYTES = 48ll << 20; /* weight bytes above which 16 M tiles share a group */
 constexpr uint32_t SUSPEND_NS = 1000000u;
+/* K steps expanded per pass (1 or 2): two K steps per fence and barrier
+ * round measured 1.42 ms against 1.64 ms for one at the Q-projection shape */
+constexpr int PASS_STEPS = 2;
+static_assert(PASS_STEPS == 1 || PASS_STEPS == 2, "pass of one or two K steps");
 constexpr uint32_t ST_TIMEOUT = 1u;
 
 __device__ unsigned int g_nv_status = 0;
@@ -222,8 +226,8 @@ __device__ __forceinline__ void scale_pairs2(uint32_t d, uint32_t &lo, uint32_t 
 }
 
 /*
- * One thread, half a row (32 elements), the NS (1 or 2) 64-wide K steps of
- * one code stage.  Step j reads the 16-byte code chunk 2 j + h of the row's
+ * One thread, half a row (32 elements), NS (1 or 2) 64-wide K steps of one
+ * code stage, from step j0.  Step j reads the 16-byte code chunk 2 j + h of the row's
  * 64-byte code line (64-byte swizzle: chunk ^ ((row / 2) % 4)) and the
  * scale bytes 2h, 2h + 1 of the row's word in atom j, and writes 32 FP16
  * values as chunks 4h .. 4h + 3 of the row in step j's operand slot
@@ -231,17 +235,17 @@ __device__ __forceinline__ void scale_pairs2(uint32_t d, uint32_t &lo, uint32_t 
  */
 template <int NS>
 __device__ __forceinline__ void expand_half_row(uint32_t code_row, uint32_t xc, uint32_t sf_word_addr,
-                                                bool have_scales, int h, uint32_t f16_row0, uint32_t f16_row1,
-                                                uint32_t xf)
+                                                bool have_scales, int j0, int h, uint32_t f16_row0,
+                                                uint32_t f16_row1, uint32_t xf)
 {
     uint4 c[NS];
     uint32_t sw[NS];
 #pragma unroll
     for (int j = 0; j < NS; ++j)
-        c[j] = ld_shared_v4(code_row + ((((uint32_t)(2 * j + h)) ^ xc) << 4));
+        c[j] = ld_shared_v4(code_row + ((((uint32_t)(2 * (j0 + j) + h)) ^ xc) << 4));
 #pragma unroll
     for (int j = 0; j < NS; ++j)
-        sw[j] = have_scales ? ld_shared_u32(sf_word_addr + (uint32_t)j * 512u) : 0u;
+        sw[j] = have_scales ? ld_shared_u32(sf_word_addr + (uint32_t)(j0 + j) * 512u) : 0u;
 #pragma unroll
     for (int j = 0; j < NS; ++j) {
         uint32_t s_lo, s_hi;
@@ -511,7 +515,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             tile_coords(t, p.num_m, p.num_n, p.raster, mb, nb);
             const int row_block = op ? nb * TILE_N + (int)(rank * 128u) : mb * TILE_M + (int)(rank * 128u);
             const bool have_scales = row_block < (op ? p.N : p.M);
-            /* one pass per code stage: its two K steps (one at an odd end) */
+            /* PASS_STEPS K steps per pass (one at an odd end) */
             for (int kb = 0; kb < KB;) {
                 if (pending && kb == FS) {
                     pending = false;
@@ -520,10 +524,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                         break;
                     }
                 }
-                const int ns = kb + 1 < KB ? 2 : 1;
+                const int ns = (PASS_STEPS == 2 && kb + 1 < KB) ? 2 : 1;
+                const int j0 = kb % SUB;
                 const uint32_t rs = ir % RS;
                 const uint32_t s0 = it % FS, s1 = (it + 1) % FS;
-                if (!warp_wait(bar_rfull + 8 * rs, (ir / RS) & 1u, lim, abort_flag) ||
+                if ((j0 == 0 && !warp_wait(bar_rfull + 8 * rs, (ir / RS) & 1u, lim, abort_flag)) ||
                     !warp_wait(bar_empty + 8 * s0, ((it / FS) & 1u) ^ 1u, lim, abort_flag) ||
                     (ns == 2 && !warp_wait(bar_empty + 8 * s1, (((it + 1) / FS) & 1u) ^ 1u, lim, abort_flag))) {
                     ok = false;
@@ -532,10 +537,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t code_row = code_base + rs * CODE_BYTES;
                 const uint32_t sf_addr = sf_base + rs * SF_BYTES;
                 if (ns == 2)
-                    expand_half_row<2>(code_row, xc, sf_addr, have_scales, h, f16_base + s0 * TILE_BYTES,
+                    expand_half_row<2>(code_row, xc, sf_addr, have_scales, 0, h, f16_base + s0 * TILE_BYTES,
                                        f16_base + s1 * TILE_BYTES, xf);
                 else
-                    expand_half_row<1>(code_row, xc, sf_addr, have_scales, h, f16_base + s0 * TILE_BYTES, 0u, xf);
+                    expand_half_row<1>(code_row, xc, sf_addr, have_scales, j0, h, f16_base + s0 * TILE_BYTES, 0u,
+                                       xf);
                 fence_proxy_async_smem(); /* generic-proxy stores -> visible to the tensor core */
                 __syncwarp();
                 if (lane == 0) {
@@ -548,9 +554,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                     mbar_arrive_cluster(mapa_shared(bar_full + 8 * s0, 0u));
                     if (ns == 2)
                         mbar_arrive_cluster(mapa_shared(bar_full + 8 * s1, 0u));
-                    mbar_arrive(bar_rempty + 8 * rs);
                 }
-                ++ir;
+                if (j0 + ns == SUB || kb + ns == KB) { /* code stage consumed */
+                    if (lane == 0)
+                        mbar_arrive(bar_rempty + 8 * rs);
+                    ++ir;
+                }
                 kb += ns;
                 it += (uint32_t)ns;
             }
