@@ -51,7 +51,7 @@ def parse(argv=None):
     ap.add_argument("--unfused", action="store_true",
                     help="chained workloads: separate q/k/v (and text k/v) GEMMs, and ffn.net.0.proj writes "
                          "BF16 with GELU + quantization as separate kernels (default: fused)")
-    ap.add_argument("--scheme", choices=["mxfp8", "fp8rowwise"], default="mxfp8",
+    ap.add_argument("--scheme", choices=["mxfp8", "fp8rowwise", "nvfp4"], default="mxfp8",
                     help="quantization scheme of the single-linear workloads (default: MXFP8)")
     ap.add_argument("--graph", action="store_true",
                     help="capture one step as a CUDA graph and time its replays (per-kernel times then "
@@ -202,6 +202,11 @@ class LinearWorkload:
 
     long_step = False
     scheme = "mxfp8"
+    gemm_kernel = "mxfp8_gemm_kernel"
+    quant_kernel = "mx_quantize_kernel"
+    profile_kernel = "mxfp8_gemm"          # kernel files the profile summary is tied to
+    tc_over_bf16 = FP8_OVER_BF16          # tensor-core rate of the GEMM's operand type vs BF16
+    dtype = "e4m3 (MXFP8 operands, fp32 accumulate, bf16 out)"
 
     def __init__(self, name, M, K, N, seed, desc):
         self.name, self.M, self.K, self.N, self.seed, self.desc = name, M, K, N, seed, desc
@@ -270,6 +275,8 @@ class FP8RowwiseLinearWorkload(LinearWorkload):
     and per output channel; Y = BF16(sx sw (Xq . Wq^T) + b)."""
 
     scheme = "fp8rowwise"
+    quant_kernel = "fp8_rowwise_quantize_bulk_kernel"
+    dtype = "e4m3 (per-channel FP8 operands, fp32 accumulate, bf16 out)"
 
     def config(self):
         return {"M": self.M, "K": self.K, "N": self.N,
@@ -306,6 +313,62 @@ class FP8RowwiseLinearWorkload(LinearWorkload):
 
     def e2e_workspace(self, dev):
         return torch.empty(self.mx.fp8rw_linear_workspace_bytes(self.M, self.K), dtype=torch.uint8, device=dev)
+
+
+class NVFP4LinearWorkload(LinearWorkload):
+    """One NVFP4 linear: E2M1 codes with a UE4M3 scale per 16 elements and
+    an FP32 global scale per tensor; Y = BF16(alpha (Xh . Wh^T) + b) with
+    alpha = 1 / (g_x g_w).  The weights' global scale comes from their amax
+    and the activations' from the amax of this workload's input, both
+    before timing (the activation scale is a calibrated constant of the
+    layer, not computed per step)."""
+
+    scheme = "nvfp4"
+    gemm_kernel = "nvfp4_gemm_kernel"
+    quant_kernel = "nvfp4_quantize_kernel"
+    profile_kernel = "nvfp4_gemm"
+    tc_over_bf16 = 1.0    # the codes are expanded to FP16: the FP16 tensor-core rate (= BF16)
+    dtype = "e2m1 + ue4m3/16 (NVFP4 operands expanded exactly to fp16 for the tensor core), fp32 accumulate, " \
+            "bf16 out"
+
+    def config(self):
+        return {"M": self.M, "K": self.K, "N": self.N,
+                "scheme": "NVFP4 (E2M1, UE4M3 scale per 16, FP32 global scale per tensor)"}
+
+    def quant_bytes(self):
+        return self.M * self.K * 2 + self.M * self.K // 2 + self.M * self.K // 16
+
+    def gemm_bytes(self):
+        M, K, N = self.M, self.K, self.N
+        return (M + N) * K * (1 / 2 + 1 / 16) + 2 * M * N + 2 * N
+
+    def setup(self, dev):
+        from mxfp8_w8a8_quantized_b200 import mxfp8, synth
+        self.mx = mxfp8
+        M, K, N, s = self.M, self.K, self.N, self.seed
+        self.x = synth.activations_device(M, K, s, 0, dev)
+        w = synth.weights_device(N, K, s, 0, dev)
+        self.b = synth.bias_device(N, s, 0, dev)
+        self.gw = mxfp8.nvfp4_global_scale(mxfp8.nvfp4_amax(w).item())
+        self.gx = mxfp8.nvfp4_global_scale(mxfp8.nvfp4_amax(self.x).item())
+        self.alpha = mxfp8.nvfp4_alpha(self.gx, self.gw)
+        self.wq, self.ws = mxfp8.nvfp4_quantize_weight(w, self.gw)   # offline weight quantization
+        del w
+        self.xq = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+        self.xs = torch.empty(mxfp8.nvfp4_scale_bytes(M, K), dtype=torch.uint8, device=dev)
+        self.y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        self.launches = 2
+
+    def step(self, T):
+        mx = self.mx
+        T("quant", mx.nvfp4_quantize, self.x, self.gx, codes=self.xq, scales=self.xs)
+        T("gemm", mx.nvfp4_gemm, self.xq, self.xs, self.wq, self.ws, self.alpha, self.b, out=self.y)
+
+    def e2e_step(self, x_dev, y_dev, ws):
+        self.mx.nvfp4_linear(x_dev, self.gx, self.wq, self.ws, self.gw, self.b, out=y_dev, workspace=ws)
+
+    def e2e_workspace(self, dev):
+        return torch.empty(self.mx.nvfp4_linear_workspace_bytes(self.M, self.K), dtype=torch.uint8, device=dev)
 
 
 class FFNPairWorkload(LinearWorkload):
@@ -451,11 +514,12 @@ class BlocksWorkload(LinearWorkload):
 
 def make_workload(name, fused=True, scheme="mxfp8"):
     from mxfp8_w8a8_quantized_b200 import synth
-    if scheme == "fp8rowwise":
+    if scheme in ("fp8rowwise", "nvfp4"):
         wl = make_workload(name)
         if type(wl) is not LinearWorkload:
-            raise ValueError("the per-channel FP8 scheme is measured on the single-linear workloads")
-        return FP8RowwiseLinearWorkload(wl.name, wl.M, wl.K, wl.N, wl.seed, wl.desc)
+            raise ValueError(f"the {scheme} scheme is measured on the single-linear workloads")
+        cls = FP8RowwiseLinearWorkload if scheme == "fp8rowwise" else NVFP4LinearWorkload
+        return cls(wl.name, wl.M, wl.K, wl.N, wl.seed, wl.desc)
     H, F = synth.HIDDEN, synth.FFN
     M1, M2, T = synth.TOKENS_480P, synth.TOKENS_832x1104, synth.TEXT_TOKENS
     if name == "c0_small":
@@ -534,7 +598,7 @@ def run_ours(args, ranks, dev):
     # a single linear is a kernel timed on its own (burst peak); the chained
     # workloads keep the GPU busy for the whole step (sustained peak)
     kind = "sustained" if wl.long_step else "burst"
-    fp8_peak = (bf16_sustained if wl.long_step else bf16_burst) * FP8_OVER_BF16
+    tc_peak = (bf16_sustained if wl.long_step else bf16_burst) * wl.tc_over_bf16
     tot = T.totals()
     g_n, g_ms = tot["gemm"]
     q_n, q_ms = tot["quant"]
@@ -551,21 +615,23 @@ def run_ours(args, ranks, dev):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "e4m3 (MXFP8 operands, fp32 accumulate, bf16 out)",
+        "dtype": wl.dtype,
         "data": "synthetic (seeded N(0,1) activations with 1% x20 outlier channels, N(0,1/sqrt(K)) weights, "
                 "N(0,0.01) f16 bias)",
         "config": dict(workload=wl.name, desc=wl.desc, **wl.config(),
                        l2="flushed between timed steps (256 MiB write outside the step events)",
                        launch="one CUDA graph per step" if graph is not None else "eager launches",
                        parallelism=f"replicas x{ranks.world}" if ranks.world > 1 else "single GPU"),
-        "roofline": {"bound": "tensor", "kernel": "mxfp8_gemm_kernel",
-                     "achieved": round(gemm_tflops, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
-                     "frac": round(gemm_tflops / fp8_peak, 4),
-                     "peak_source": f"{peak_src} bf16 {kind} x {FP8_OVER_BF16} (nominal FP8/BF16 ratio)",
-                     "traffic": load_traffic(wl.profile_key),
+        "roofline": {"bound": "tensor", "kernel": wl.gemm_kernel,
+                     "achieved": round(gemm_tflops, 1), "peak": round(tc_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(gemm_tflops / tc_peak, 4),
+                     "peak_source": (f"{peak_src} bf16 {kind} x {FP8_OVER_BF16} (nominal FP8/BF16 ratio)"
+                                     if wl.tc_over_bf16 != 1.0 else
+                                     f"{peak_src} bf16 {kind} (the FP16 kind runs at the BF16 rate)"),
+                     "traffic": load_traffic(wl.profile_key, wl.profile_kernel),
                      "algorithmic_bytes_per_step": round(wl.gemm_bytes()),
                      "launches_per_step": g_n // kernel_steps, "avg_launch_ms": round(g_ms / g_n, 4)},
-        "quant": {"kernel": "mx_quantize_kernel", "achieved_gbs": round(quant_gbs, 1), "peak_gbs": hbm,
+        "quant": {"kernel": wl.quant_kernel, "achieved_gbs": round(quant_gbs, 1), "peak_gbs": hbm,
                   "frac": round(quant_gbs / hbm, 4), "peak_source": f"{peak_src} copy",
                   "bytes_per_step": wl.quant_bytes(), "launches_per_step": q_n // kernel_steps,
                   "avg_launch_ms": round(q_ms / q_n, 4)},
@@ -616,15 +682,15 @@ def run_e2e(args, wl, ranks, dev):
             "ms_per_step": round(ms / steps, 3)}
 
 
-def load_traffic(workload):
+def load_traffic(workload, kernel="mxfp8_gemm"):
     """DRAM bytes per GEMM launch from the committed ncu summary
-    (profiles/mxfp8_gemm_<workload>.json), if it was taken on the current
-    kernel sources; else None."""
-    path = os.path.join(ROOT, "profiles", f"mxfp8_gemm_{workload}.json")
+    (profiles/<kernel>_<workload>.json), if it was taken on the kernel's
+    current source files; else None."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.json")
     try:
         d = json.load(open(path))
         from mxfp8_w8a8_quantized_b200 import build
-        if d.get("kernel_source_sha") != build.source_sha():
+        if d.get("kernel_source_sha") != build.source_sha(kernel):
             return None
         return d["dram_bytes_per_launch"]
     except Exception:
@@ -643,12 +709,18 @@ def oracle_sample(wl, rows):
     x = synth.activations(rows, wl.K, wl.seed, index=100)
     w = synth.weights(wl.N, wl.K, wl.seed, index=100)
     b = synth.bias(wl.N, wl.seed, index=100)
-    if wl.scheme == "fp8rowwise":
-        wq, ws = oracle.quantize_rowwise_f32(w.numpy())
-    else:
-        wq, ws = oracle.quantize_f32(w.numpy())
     xb = x.view(torch.int16).numpy().view(np.uint16)
     bb = b.view(torch.int16).numpy().view(np.uint16)
+    if wl.scheme == "fp8rowwise":
+        wq, ws = oracle.quantize_rowwise_f32(w.numpy())
+    elif wl.scheme == "nvfp4":
+        wb = w.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        gw = oracle.nvfp4_global_scale(np.abs(w.to(torch.bfloat16).float().numpy()).max())
+        gx = oracle.nvfp4_global_scale(np.abs(x.float().numpy()).max())
+        wq, ws = oracle.nvfp4_quantize_bf16(wb, gw)
+        return xb, (wq, ws, gx, gw), None, bb, wl.scheme
+    else:
+        wq, ws = oracle.quantize_f32(w.numpy())
     return xb, wq, ws, bb, wl.scheme
 
 
@@ -658,6 +730,10 @@ def oracle_step(xb, wq, ws, bb, scheme):
     if scheme == "fp8rowwise":
         xq, xs = oracle.quantize_rowwise_bf16(xb)
         return oracle.linear_rowwise(xq, xs, wq, ws, bb)
+    if scheme == "nvfp4":
+        wq4, ws4, gx, gw = wq
+        xq, xs = oracle.nvfp4_quantize_bf16(xb, gx)
+        return oracle.nvfp4_linear(xq, xs, gx, wq4, ws4, gw, bb)
     xq, xs = oracle.quantize_bf16(xb)
     return oracle.linear(xq, xs, wq, ws, bb)
 
@@ -729,7 +805,7 @@ def chain_oracle_sample(wl):
 
 def cpu_baseline(wl, target_s):
     import oracle
-    if type(wl) not in (LinearWorkload, FP8RowwiseLinearWorkload):
+    if type(wl) not in (LinearWorkload, FP8RowwiseLinearWorkload, NVFP4LinearWorkload):
         # chained: grow the row sample until one pass takes about target_s
         make = chain_oracle_sample(wl)
         rows = 2
@@ -762,7 +838,7 @@ def run_reference(args, ranks):
     """The oracle as the reference arm: CPU, rank 0 only."""
     import oracle
     wl = make_workload(args.workload, scheme=args.scheme)
-    if type(wl) not in (LinearWorkload, FP8RowwiseLinearWorkload):
+    if type(wl) not in (LinearWorkload, FP8RowwiseLinearWorkload, NVFP4LinearWorkload):
         wl = LinearWorkload(wl.name, wl.M, wl.K, wl.K, wl.seed, wl.desc + " (first linear only)")
     if ranks.rank != 0:
         return None

@@ -101,3 +101,26 @@ def test_fused_accounting():
     bp = bench.make_workload("c3_block_832x1104", fused=False)
     assert bp.quant_bytes() - bf.quant_bytes() == M * F * 3 + M * F // 32
     assert bf.flops() == bp.flops()
+
+
+@pytest.mark.parametrize("scheme", ["fp8rowwise", "nvfp4"])
+def test_reference_arm_other_schemes(scheme):
+    r = _bench(["--impl", "reference", "--workload", "c0_small", "--scheme", scheme, "--steps", "2",
+                "--warmup", "1", "--reference-seconds", "3"], {})
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads(r.stdout.strip().splitlines()[-1])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["config"]["scheme"]
+
+
+def test_nvfp4_accounting():
+    """NVFP4 moves 4-bit codes plus one scale byte per 16 elements."""
+    sys.path.insert(0, ROOT)
+    import bench
+    wl = bench.make_workload("c1_q_proj_480p", scheme="nvfp4")
+    M, K, N = 32760, 5120, 5120
+    assert wl.flops() == 2.0 * M * N * K
+    assert wl.quant_bytes() == M * K * 2 + M * K // 2 + M * K // 16
+    assert wl.gemm_bytes() == pytest.approx((M + N) * K * 9 / 16 + 2 * M * N + 2 * N)
+    assert wl.tc_over_bf16 == 1.0 and wl.profile_kernel == "nvfp4_gemm"
+    with pytest.raises(ValueError):
+        bench.make_workload("c2_ffn_pair_832x1104", scheme="nvfp4")
