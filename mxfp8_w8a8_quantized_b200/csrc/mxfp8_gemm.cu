@@ -124,7 +124,7 @@ struct Cfg {
     static constexpr uint32_t OFF_EPI = OFF_SFB + STAGES * SFB_BYTES; /* 1 KiB aligned */
     static constexpr uint32_t EPI_BUF = 32 * 32 * 2;                    /* 32 rows x 32 BF16 */
     static constexpr uint32_t OFF_BAR = OFF_EPI + EPI_WARPS * EPI_BUF;
-    static constexpr uint32_t NUM_BARS = 3 * STAGES + 3; /* full[], empty[], sf_full[], tmem_full, tmem_empty, drain */
+    static constexpr uint32_t NUM_BARS = 3 * STAGES + 5; /* full[], empty[], sf_full[], tmem_full[2], tmem_empty[2], drain */
     static constexpr uint32_t OFF_TMEMPTR = OFF_BAR + NUM_BARS * 8;
     static constexpr uint32_t OFF_ABORT = OFF_TMEMPTR + 4;
     static constexpr uint32_t SMEM_USED = OFF_TMEMPTR + 16;
@@ -422,9 +422,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const uint32_t bar_full = sbase + C::OFF_BAR;          /* + 8 s */
     const uint32_t bar_empty = bar_full + C::STAGES * 8;   /* + 8 s */
     const uint32_t bar_sffull = bar_empty + C::STAGES * 8; /* + 8 s */
-    const uint32_t bar_tfull = bar_sffull + C::STAGES * 8;
-    const uint32_t bar_tempty = bar_tfull + 8;
-    const uint32_t bar_drain = bar_tempty + 8;
+    const uint32_t bar_tfull = bar_sffull + C::STAGES * 8; /* + 8 b, accumulator b */
+    const uint32_t bar_tempty = bar_tfull + 2 * 8;        /* + 8 b */
+    const uint32_t bar_drain = bar_tempty + 2 * 8;
+    /* Accumulators in TMEM: with block scales the scale columns take the
+     * upper half, so one; without them (per-channel FP8) two, and the MMA
+     * runs the next tile while the epilogue drains the last.  Tile number
+     * u uses accumulator acc_buf(u) for the acc_use(u)-th time. */
+    constexpr uint32_t NACC = BS ? 1u : 2u;
+    auto acc_buf = [](uint32_t u) { return NACC == 2u ? (u & 1u) : 0u; };
+    auto acc_use = [](uint32_t u) { return NACC == 2u ? (u >> 1) : u; };
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + C::OFF_TMEMPTR);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_ABORT);
 
@@ -435,8 +442,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             mbar_init(bar_empty + 8 * s, 1);
             mbar_init(bar_sffull + 8 * s, 1);
         }
-        mbar_init(bar_tfull, 1);
-        mbar_init(bar_tempty, C::TEMPTY_ARRIVALS);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_tfull + 8 * b, 1);
+            mbar_init(bar_tempty + 8 * b, C::TEMPTY_ARRIVALS);
+        }
         mbar_init(bar_drain, 1);
         fence_mbar_init();
     }
@@ -538,7 +547,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             uint32_t it = 0, tl = 0;
             bool ok = true, any = false;
             for (int t = tile0; ok && t < num_tiles; t += tstep, ++tl) {
-                if (!wait_bounded(bar_tempty, (tl & 1u) ^ 1u, lim, abort_flag)) {
+                const uint32_t ab = acc_buf(tl);
+                const uint32_t tacc = tmem + ACC_COL + 256u * ab;
+                if (!wait_bounded(bar_tempty + 8 * ab, (acc_use(tl) & 1u) ^ 1u, lim, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -565,10 +576,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
                         for (int k = 0; k < BK / 32; ++k) {
                             if constexpr (PAIR)
-                                tc_mma_f8_pair(tmem + ACC_COL, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k),
+                                tc_mma_f8_pair(tacc, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k),
                                                idesc, (kb | k) != 0);
                             else
-                                tc_mma_f8(tmem + ACC_COL, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc,
+                                tc_mma_f8(tacc, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc,
                                           (kb | k) != 0);
                         }
                         if constexpr (PAIR)
@@ -581,7 +592,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         (void)sfb_s;
 #pragma unroll
                         for (int k = 0; k < BK / 32; ++k)
-                            tc_mma_mxf8_pair(tmem + ACC_COL, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k),
+                            tc_mma_mxf8_pair(tacc, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k),
                                              idesc_with_sf_id(idesc, (uint32_t)k), tsfa, tsfb, (kb | k) != 0);
                         tc_commit_pair(bar_empty + 8 * s, (uint16_t)0x3);
                     } else {
@@ -590,7 +601,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         tc_cp_32x128b_warpx4(tsfb + 4, desc_sf_32x16(sfb_s + 512u));
 #pragma unroll
                         for (int k = 0; k < BK / 32; ++k)
-                            tc_mma_mxf8(tmem + ACC_COL, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k),
+                            tc_mma_mxf8(tacc, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k),
                                         idesc_with_sf_id(idesc, (uint32_t)k), tsfa, tsfb, (kb | k) != 0);
                         tc_commit(bar_empty + 8 * s);
                     }
@@ -599,14 +610,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 if (!ok)
                     break;
                 if constexpr (PAIR)
-                    tc_commit_pair(bar_tfull, (uint16_t)0x3);
+                    tc_commit_pair(bar_tfull + 8 * ab, (uint16_t)0x3);
                 else
-                    tc_commit(bar_tfull);
+                    tc_commit(bar_tfull + 8 * ab);
             }
-            if (ok && tl > 0) {
+            if (ok) {
                 /* every epilogue (the peer's included) has released the last
-                 * accumulator, so no remote arrival is still in flight */
-                (void)wait_bounded(bar_tempty, (tl & 1u) ^ 1u, lim, abort_flag);
+                 * accumulators, so no remote arrival is still in flight */
+                for (uint32_t u = tl > NACC ? tl - NACC : 0u; u < tl; ++u)
+                    (void)wait_bounded(bar_tempty + 8 * acc_buf(u), acc_use(u) & 1u, lim, abort_flag);
             }
             if (!ok && any) {
                 /* wait for this thread's MMAs and copies before TMEM is freed */
@@ -651,26 +663,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         /* ------------------------------------------------ epilogue */
         const int q = warp & 3;            /* TMEM sub-partition this warp may read */
         const int h = (warp - 2) >> 2;     /* column half of the 256-wide tile */
-        const uint32_t tempty_lead = PAIR ? mapa_shared(bar_tempty, 0u) : bar_tempty;
         uint32_t tl = 0;
         for (int t = tile0; t < num_tiles; t += tstep, ++tl) {
             int mb, nb;
             tile_coords(t, p.num_m, p.num_n, p.raster, mb, nb);
             /* every lane polls; the vote keeps the warp converged for the
              * .sync.aligned TMEM load and makes the outcome warp-uniform */
-            const bool got = wait_bounded(bar_tfull, tl & 1u, lim, abort_flag, SUSPEND_EPI);
+            const uint32_t ab = acc_buf(tl);
+            const bool got = wait_bounded(bar_tfull + 8 * ab, acc_use(tl) & 1u, lim, abort_flag, SUSPEND_EPI);
             if (!__all_sync(0xFFFFFFFFu, got))
                 break;
             tc_fence_after();
             uint32_t acc[128];
-            tmem_ld_32x32b_x128_sync(tmem + ((uint32_t)(32 * q) << 16) + ACC_COL + (uint32_t)(h * 128), acc);
+            tmem_ld_32x32b_x128_sync(tmem + ((uint32_t)(32 * q) << 16) + ACC_COL + 256u * ab + (uint32_t)(h * 128),
+                                     acc);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
                 if constexpr (PAIR)
-                    mbar_arrive_cluster(tempty_lead);
+                    mbar_arrive_cluster(mapa_shared(bar_tempty + 8 * ab, 0u));
                 else
-                    mbar_arrive(bar_tempty);
+                    mbar_arrive(bar_tempty + 8 * ab);
             }
 
             const int row0 = mb * C::TILE_M + (int)(rank * 128u) + 32 * q;
