@@ -93,6 +93,7 @@ constexpr uint32_t SUSPEND_PIPE = MX_SUSPEND_PIPE;
 constexpr uint32_t SUSPEND_EPI = MX_SUSPEND_EPI;
 constexpr int PREFETCH_KB = MX_PREFETCH_KB; /* K steps the L2 prefetch runs ahead of the loads (0 = off) */
 constexpr uint32_t ST_TIMEOUT = 1u;
+constexpr uint64_t ABORT_SETTLE_NS = 200000; /* after a timeout: time for in-flight copies to land */
 
 /* What the epilogue writes. */
 enum EpiMode : int {
@@ -704,6 +705,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        /* a wait gave up: copies this CTA issued may still be landing in its
+         * shared memory; let them settle (bounded) before the CTA exits */
+        if (threadIdx.x == 0) {
+            const uint64_t t0 = globaltimer_ns();
+            while (globaltimer_ns() - t0 < ABORT_SETTLE_NS)
+                __nanosleep(1000);
+        }
+        __syncthreads();
+    }
     if constexpr (PAIR)
         cluster_sync_all(); /* neither CTA leaves while the pair may still touch it */
     tc_fence_after();

@@ -99,6 +99,7 @@ constexpr uint32_t SUSPEND_NS = 1000000u;
 constexpr int PASS_STEPS = 2;
 static_assert(PASS_STEPS == 1 || PASS_STEPS == 2, "pass of one or two K steps");
 constexpr uint32_t ST_TIMEOUT = 1u;
+constexpr uint64_t ABORT_SETTLE_NS = 200000; /* after a timeout: time for in-flight copies to land */
 
 __device__ unsigned int g_nv_status = 0;
 
@@ -583,6 +584,16 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        /* a wait gave up: copies this CTA issued may still be landing in its
+         * shared memory; let them settle (bounded) before the CTA exits */
+        if (threadIdx.x == 0) {
+            const uint64_t t0 = globaltimer_ns();
+            while (globaltimer_ns() - t0 < ABORT_SETTLE_NS)
+                __nanosleep(1000);
+        }
+        __syncthreads();
+    }
     cluster_sync_all(); /* neither CTA leaves while the pair may still touch it */
     tc_fence_after();
     if (warp == 1) {
