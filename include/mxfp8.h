@@ -222,6 +222,23 @@ mxfp8_status mxfp8_linear_noalloc(const void *X, int64_t M, int64_t K,
  */
 mxfp8_status mxfp8_device_status(mxfp8_stream_t stream);
 
+/* Which kernel family's bounded wait mxfp8_selftest_wait_timeout exercises. */
+typedef enum {
+    MXFP8_SELFTEST_GEMM = 0,           /* the MXFP8 / per-channel FP8 GEMM */
+    MXFP8_SELFTEST_NVFP4_GEMM = 1,     /* the NVFP4 GEMM */
+    MXFP8_SELFTEST_ROWWISE_QUANT = 2   /* the per-channel FP8 activation quantizer */
+} mxfp8_selftest;
+
+/*
+ * Failure-path self-test: launches one thread that waits, with that kernel
+ * family's bounded wait, on an mbarrier that nothing arrives at.  After
+ * timeout_ns (1 .. 10^10) the wait gives up and records the timeout in the
+ * status word, so the next mxfp8_device_status() returns MXFP8_ERR_TIMEOUT
+ * (and clears it) while the context stays usable.  Nothing else is in flight
+ * in the test kernel.  Bad `which` or timeout: MXFP8_ERR_ARG.
+ */
+mxfp8_status mxfp8_selftest_wait_timeout(int which, uint64_t timeout_ns, mxfp8_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

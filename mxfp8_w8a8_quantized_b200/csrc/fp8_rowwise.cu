@@ -120,6 +120,19 @@ __device__ __forceinline__ bool rw_wait(uint32_t bar, uint32_t parity, unsigned 
     return true;
 }
 
+/* Self-test of rw_wait: a wait on an mbarrier that nothing arrives at gives
+ * up after limit_ns; the kernel records it as the quantizer does. */
+__global__ void rw_wait_selftest_kernel(unsigned long long limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        fence_mbar_init();
+        if (!rw_wait(smem_u32(&bar), 0u, limit_ns))
+            atomicOr(&g_rw_status, 1u);
+    }
+}
+
 __global__ void __launch_bounds__(RWB_WARPS * 32, 1) fp8_rowwise_quantize_bulk_kernel(
     const uint16_t *__restrict__ X, int64_t M, int K, int64_t ldx, uint8_t *__restrict__ Q, float *__restrict__ S,
     int ns, uint32_t slot_bytes, unsigned long long timeout_ns)
@@ -332,6 +345,12 @@ cudaError_t launch_fp8_rowwise_quantize(const void *X, bool f32_in, int64_t M, i
 }
 
 /* Reads and clears the row-wise quantizer's status word (synchronous). */
+cudaError_t launch_rw_wait_selftest(unsigned long long limit_ns, cudaStream_t stream)
+{
+    rw_wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns);
+    return cudaGetLastError();
+}
+
 cudaError_t read_and_clear_rw_status(unsigned int *out)
 {
     unsigned int zero = 0;

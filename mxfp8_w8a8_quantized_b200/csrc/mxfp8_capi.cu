@@ -27,6 +27,9 @@ int launch_nvfp4_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, cons
                       int64_t N, float alpha, const void *bias, void *Y, cudaStream_t stream,
                       unsigned long long timeout_ns, cudaError_t *err);
 cudaError_t read_and_clear_nv_status(unsigned int *out);
+cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t stream);
+cudaError_t launch_nv_wait_selftest(unsigned long long limit_ns, cudaStream_t stream);
+cudaError_t launch_rw_wait_selftest(unsigned long long limit_ns, cudaStream_t stream);
 } // namespace mx
 
 namespace {
@@ -428,6 +431,23 @@ mxfp8_status nvfp4_linear(const void *X, int64_t M, int64_t K, float x_global_sc
     if (st != MXFP8_OK)
         return st;
     return nvfp4_gemm(codes, scales, M, K, Wq, Wscale, N, (float)a, bias, Y, stream);
+}
+
+mxfp8_status mxfp8_selftest_wait_timeout(int which, uint64_t timeout_ns, mxfp8_stream_t stream)
+{
+    if (timeout_ns == 0 || timeout_ns > 10000000000ull)
+        return MXFP8_ERR_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    switch (which) {
+    case MXFP8_SELFTEST_GEMM:
+        return from_cuda(mx::launch_wait_selftest(timeout_ns, s));
+    case MXFP8_SELFTEST_NVFP4_GEMM:
+        return from_cuda(mx::launch_nv_wait_selftest(timeout_ns, s));
+    case MXFP8_SELFTEST_ROWWISE_QUANT:
+        return from_cuda(mx::launch_rw_wait_selftest(timeout_ns, s));
+    default:
+        return MXFP8_ERR_ARG;
+    }
 }
 
 mxfp8_status mxfp8_device_status(mxfp8_stream_t stream)

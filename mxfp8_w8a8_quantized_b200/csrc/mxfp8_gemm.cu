@@ -727,6 +727,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
 }
 
+/* Self-test of the GEMM's bounded wait: one thread waits on an mbarrier
+ * that nothing arrives at; after limit_ns the wait gives up and records
+ * ST_TIMEOUT in the status word, as a stalled pipeline would.  Nothing else
+ * is in flight, so the kernel simply returns. */
+__global__ void wait_selftest_kernel(unsigned long long limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ uint32_t abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0u;
+        mbar_init(smem_u32(&bar), 1);
+        fence_mbar_init();
+        (void)wait_bounded(smem_u32(&bar), 0u, limit_ns, &abort_flag);
+    }
+}
+
 /* ------------------------------------------------------------ host side */
 /* K-major E4M3 operand [rows, K]: box 128 (K bytes) x box_rows, 128-byte swizzle. */
 static bool make_operand_map(CUtensorMap *m, const void *base, int64_t rows, int64_t K, uint32_t box_rows)
@@ -962,6 +978,12 @@ int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void
         return 2;
     }
     return 0;
+}
+
+cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t stream)
+{
+    wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns);
+    return cudaGetLastError();
 }
 
 /* Reads and clears the status word of the current device (synchronous). */

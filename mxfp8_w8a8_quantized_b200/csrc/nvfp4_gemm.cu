@@ -602,6 +602,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 }
 
+/* Self-test of the bounded wait used by this kernel (as in the MXFP8 GEMM):
+ * a wait on an mbarrier that nothing arrives at gives up after limit_ns and
+ * records ST_TIMEOUT. */
+__global__ void wait_selftest_kernel(unsigned long long limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ uint32_t abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0u;
+        mbar_init(smem_u32(&bar), 1);
+        fence_mbar_init();
+        (void)wait_bounded(smem_u32(&bar), 0u, limit_ns, &abort_flag);
+    }
+}
+
 /* ------------------------------------------------------------ host side */
 struct DevInfo {
     bool init = false;
@@ -707,6 +722,12 @@ int launch_nvfp4_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, cons
         return 2;
     }
     return 0;
+}
+
+cudaError_t launch_nv_wait_selftest(unsigned long long limit_ns, cudaStream_t stream)
+{
+    nv::wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns);
+    return cudaGetLastError();
 }
 
 /* Reads and clears the NVFP4 GEMM's status word (synchronous). */

@@ -71,6 +71,8 @@ _lib.nvfp4_linear_workspace_bytes.argtypes = [_I64, _I64]
 _lib.nvfp4_linear_workspace_bytes.restype = _SZ
 _lib.nvfp4_linear.argtypes = [_P, _I64, _I64, _F, _P, _P, _I64, _F, _P, _P, _P, _SZ, _P]
 _lib.nvfp4_linear.restype = ctypes.c_int
+_lib.mxfp8_selftest_wait_timeout.argtypes = [ctypes.c_int, ctypes.c_uint64, _P]
+_lib.mxfp8_selftest_wait_timeout.restype = ctypes.c_int
 _lib.mxfp8_device_status.argtypes = [_P]
 _lib.mxfp8_device_status.restype = ctypes.c_int
 
@@ -82,7 +84,7 @@ ACT_GELU_TANH = 1
 EXPORTS = ("mxfp8_status_str", "mxfp8_scale_bytes", "mxfp8_quantize", "mxfp8_quantize_weight_f32",
            "mxfp8_linear_workspace_bytes", "mxfp8_linear", "mxfp8_gemm_prequant",
            "mxfp8_gelu_tanh_bf16", "mxfp8_device_status", "mxfp8_linear_noalloc",
-           "mxfp8_gemm_quantize_out",
+           "mxfp8_gemm_quantize_out", "mxfp8_selftest_wait_timeout",
            "fp8rw_quantize_bf16", "fp8rw_quantize_weight_f32", "fp8rw_gemm", "fp8rw_linear_workspace_bytes",
            "fp8rw_linear",
            "nvfp4_scale_bytes", "nvfp4_amax_bf16", "nvfp4_amax_f32", "nvfp4_quantize_bf16",
@@ -368,6 +370,15 @@ def nvfp4_linear(x: torch.Tensor, x_global_scale: float, wq, wscale, w_global_sc
     _check(_lib.nvfp4_linear(_ptr(x), M, K, x_global_scale, _ptr(wq), _ptr(wscale), N, w_global_scale, _ptr(bias),
                              _ptr(out), _ptr(workspace), workspace.numel(), _stream()), "nvfp4_linear")
     return out
+
+
+SELFTEST_GEMM, SELFTEST_NVFP4_GEMM, SELFTEST_ROWWISE_QUANT = 0, 1, 2
+
+
+def selftest_wait_timeout(which: int, timeout_ns: int) -> None:
+    """Launch the bounded-wait self-test of one kernel family: the next
+    device_status() reports MXFP8_ERR_TIMEOUT."""
+    _check(_lib.mxfp8_selftest_wait_timeout(which, timeout_ns, _stream()), "mxfp8_selftest_wait_timeout")
 
 
 def device_status() -> int:

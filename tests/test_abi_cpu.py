@@ -200,3 +200,13 @@ def test_binding_checks_every_status_with_its_entry_name():
         assert isinstance(status, ast.Call) and isinstance(name, ast.Constant)
         if isinstance(status.func, ast.Attribute):      # _lib.<entry>(...); else a chosen entry
             assert status.func.attr == name.value, ast.unparse(c)[:120]
+
+
+def test_selftest_argument_checks(lib):
+    P = ctypes.c_void_p
+    lib.mxfp8_selftest_wait_timeout.argtypes = [ctypes.c_int, ctypes.c_uint64, P]
+    ARG = 1
+    assert lib.mxfp8_selftest_wait_timeout(3, 1000000, None) == ARG          # unknown kernel family
+    assert lib.mxfp8_selftest_wait_timeout(-1, 1000000, None) == ARG
+    assert lib.mxfp8_selftest_wait_timeout(0, 0, None) == ARG                # no limit
+    assert lib.mxfp8_selftest_wait_timeout(0, 20_000_000_000, None) == ARG   # above 10 s
