@@ -78,20 +78,10 @@ constexpr uint32_t ACC_COL = 0; /* 256 FP32 columns */
  * of DRAM reads per launch; the Q projection reads least with 8). */
 constexpr int RASTER_SMALL_B = 8, RASTER_LARGE_B = 16;
 constexpr int64_t RASTER_LARGE_B_BYTES = 48ll << 20;
-#ifndef MX_PREFETCH_KB
-#define MX_PREFETCH_KB 0
-#endif
-#ifndef MX_SUSPEND_PIPE
-#define MX_SUSPEND_PIPE 1000000
-#endif
-#ifndef MX_SUSPEND_EPI
-#define MX_SUSPEND_EPI 1000000
-#endif
 /* mbarrier.try_wait suspend-time hints (ns): the producer and MMA threads wait
  * briefly and often, the epilogue warps for a whole tile */
-constexpr uint32_t SUSPEND_PIPE = MX_SUSPEND_PIPE;
-constexpr uint32_t SUSPEND_EPI = MX_SUSPEND_EPI;
-constexpr int PREFETCH_KB = MX_PREFETCH_KB; /* K steps the L2 prefetch runs ahead of the loads (0 = off) */
+constexpr uint32_t SUSPEND_PIPE = 1000000;
+constexpr uint32_t SUSPEND_EPI = 1000000;
 constexpr uint32_t ST_TIMEOUT = 1u;
 constexpr uint64_t ABORT_SETTLE_NS = 200000; /* after a timeout: time for in-flight copies to land */
 
@@ -501,27 +491,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     const uint32_t dB = sbase + C::OFF_B + s * C::B_BYTES;
                     const uint32_t dSA = sbase + C::OFF_SFA + s * C::SFA_BYTES;
                     const uint32_t dSB = sbase + C::OFF_SFB + s * C::SFB_BYTES;
-                    if (PREFETCH_KB > 0) {
-                        /* operand boxes PREFETCH_KB K steps ahead (in this tile
-                         * or the next one of this CTA) go to L2 now, so that
-                         * the stage loads hit L2 instead of waiting on DRAM */
-                        int pkb = kb + PREFETCH_KB, pt = t;
-                        if (pkb >= KB) {
-                            pkb -= KB;
-                            pt += tstep;
-                        }
-                        if (pt < num_tiles && pkb < KB) {
-                            int pmb = mb, pnb = nb;
-                            if (pt != t)
-                                tile_coords(pt, p.num_m, p.num_n, p.raster, pmb, pnb);
-                            const int pra = pmb * C::TILE_M + (int)(rank * 128u);
-                            const int prb = pnb * C::TILE_N + (int)(rank * C::B_ROWS);
-                            if (pra < p.M)
-                                tma_prefetch_2d(&tmap_a, pkb * BK, pra);
-                            if (prb < p.N)
-                                tma_prefetch_2d(&tmap_b, pkb * BK, prb);
-                        }
-                    }
                     if constexpr (PAIR) {
                         const uint32_t lead = mapa_shared(full, 0u);
                         tma_load_2d_pair(dA, &tmap_a, kb * BK, rowA, lead);

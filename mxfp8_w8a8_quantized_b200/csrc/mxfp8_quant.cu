@@ -33,14 +33,8 @@
 
 namespace mx {
 
-#ifndef MX_QUNROLL
-#define MX_QUNROLL 2
-#endif
-#ifndef MX_QMINBLOCKS
-#define MX_QMINBLOCKS 1
-#endif
 constexpr int QTHREADS = 256;
-constexpr int QUNROLL = MX_QUNROLL;     /* row segments in flight per warp */
+constexpr int QUNROLL = 2;              /* row segments in flight per warp */
 
 /* 16 consecutive elements of one row: one lane's share of a row segment. */
 template <bool F32_IN>
@@ -118,7 +112,7 @@ __device__ __forceinline__ uint4 codes_seg16(const Seg16<F32_IN> &s, float m)
  * [M, Mrows) only write zero scale padding (tensor-core layout).
  */
 template <bool F32_IN, bool SF_TC>
-__global__ void __launch_bounds__(QTHREADS, MX_QMINBLOCKS) mx_quantize_kernel(const void *__restrict__ X, int64_t M,
+__global__ void __launch_bounds__(QTHREADS, 1) mx_quantize_kernel(const void *__restrict__ X, int64_t M,
                                                                               int64_t K, int64_t ldx,
                                                                               uint8_t *__restrict__ Q,
                                                                               uint8_t *__restrict__ S, int64_t Mrows,

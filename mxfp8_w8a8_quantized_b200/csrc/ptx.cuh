@@ -69,12 +69,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int3
         "l"(tmap), "r"(c0), "r"(c1), "r"(bar)
         : "memory");
 }
-/* Bring the box at (c0, c1) into L2 without waiting or landing it in smem. */
-__device__ __forceinline__ void tma_prefetch_2d(const void *tmap, int32_t c0, int32_t c1)
-{
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(tmap), "r"(c0), "r"(c1)
-                 : "memory");
-}
 /* Untiled bulk load: both addresses 16-byte aligned, bytes % 16 == 0. */
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
 {
@@ -222,11 +216,7 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t a, uint32_t rank)
 /* arrive on an mbarrier that may live in another CTA of the cluster */
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
 {
-#ifdef MX_ARRIVE_RELEASE_CLUSTER
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-#else
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-#endif
 }
 __device__ __forceinline__ void cluster_sync_all()
 {
