@@ -35,14 +35,15 @@ def check_chain(name, got, ref64, ref32):
     assert ok, (name, stats)
 
 
-OUT = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "gpurun_out")
-
-
 def record(name, **kv):
-    """Keep the observed chain distances next to the run's other outputs."""
+    """Append the observed chain distances to the file CHAIN_PARITY_LOG
+    names (JSON lines), when it is set."""
+    path = os.environ.get("CHAIN_PARITY_LOG")
+    if not path:
+        return
     try:
-        os.makedirs(OUT, exist_ok=True)
-        with open(os.path.join(OUT, "chain_parity.jsonl"), "a") as f:
+        os.makedirs(os.path.dirname(os.path.abspath(path)), exist_ok=True)
+        with open(path, "a") as f:
             f.write(json.dumps(dict(test=name, **kv)) + "\n")
     except OSError:
         pass
