@@ -375,9 +375,8 @@ mxfp8_status nvfp4_quantize_weight_f32(const float *W, int64_t N, int64_t K, flo
     return nvfp4_quantize_any(W, true, N, K, K, global_scale, Wq, Wscale, stream);
 }
 
-mxfp8_status nvfp4_gemm(const void *Xq, const void *Xscale, int64_t M, int64_t K, const void *Wq,
-                        const void *Wscale, int64_t N, float alpha, const void *bias, void *Y,
-                        mxfp8_stream_t stream)
+static mxfp8_status nvfp4_gemm_args(const void *Xq, const void *Xscale, int64_t M, int64_t K, const void *Wq,
+                                    const void *Wscale, int64_t N, float alpha, const void *bias, const void *Y)
 {
     if (M < 0 || K <= 0 || N <= 0 || !(alpha > 0.0f) || !(alpha < 3.0e38f))
         return MXFP8_ERR_ARG;
@@ -390,6 +389,16 @@ mxfp8_status nvfp4_gemm(const void *Xq, const void *Xscale, int64_t M, int64_t K
     if (!aligned(Xq, 16) || !aligned(Xscale, 16) || !aligned(Wq, 16) || !aligned(Wscale, 16) || !aligned(Y, 16) ||
         (bias && !aligned(bias, 16)))
         return MXFP8_ERR_ALIGN;
+    return MXFP8_OK;
+}
+
+mxfp8_status nvfp4_gemm(const void *Xq, const void *Xscale, int64_t M, int64_t K, const void *Wq,
+                        const void *Wscale, int64_t N, float alpha, const void *bias, void *Y,
+                        mxfp8_stream_t stream)
+{
+    mxfp8_status st = nvfp4_gemm_args(Xq, Xscale, M, K, Wq, Wscale, N, alpha, bias, Y);
+    if (st != MXFP8_OK || M == 0)
+        return st;
     cudaError_t e;
     int r = mx::launch_nvfp4_gemm(Xq, Xscale, M, K, Wq, Wscale, N, alpha, bias, Y,
                                   reinterpret_cast<cudaStream_t>(stream), kWaitLimitNs, &e);
@@ -422,15 +431,17 @@ mxfp8_status nvfp4_linear(const void *X, int64_t M, int64_t K, float x_global_sc
         return MXFP8_ERR_ALIGN;
     if (ws_bytes < nvfp4_linear_workspace_bytes(M, K))
         return MXFP8_ERR_ARG;
-    const double a = 1.0 / ((double)x_global_scale * (double)w_global_scale);
-    if (!(a > 0.0) || !(a < 3.0e38))
-        return MXFP8_ERR_ARG;
+    const float alpha = (float)(1.0 / ((double)x_global_scale * (double)w_global_scale));
     uint8_t *codes = static_cast<uint8_t *>(workspace);
     uint8_t *scales = codes + round_up((size_t)M * (size_t)(K / 2), 256);
-    mxfp8_status st = nvfp4_quantize_bf16(X, M, K, K, x_global_scale, codes, scales, stream);
+    /* every check of both steps before anything is launched */
+    mxfp8_status st = nvfp4_gemm_args(codes, scales, M, K, Wq, Wscale, N, alpha, bias, Y);
     if (st != MXFP8_OK)
         return st;
-    return nvfp4_gemm(codes, scales, M, K, Wq, Wscale, N, (float)a, bias, Y, stream);
+    st = nvfp4_quantize_bf16(X, M, K, K, x_global_scale, codes, scales, stream);
+    if (st != MXFP8_OK)
+        return st;
+    return nvfp4_gemm(codes, scales, M, K, Wq, Wscale, N, alpha, bias, Y, stream);
 }
 
 mxfp8_status mxfp8_selftest_wait_timeout(int which, uint64_t timeout_ns, mxfp8_stream_t stream)

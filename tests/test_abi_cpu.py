@@ -171,6 +171,12 @@ def test_nvfp4_gemm_argument_checks_return_before_launch(lib):
     assert L.nvfp4_linear(FAKE, 4, 96, 1.0, FAKE, FAKE, 16, 1.0, None, FAKE, FAKE, need, None) == SHAPE
     assert L.nvfp4_linear(FAKE, 4, 128, 0.0, FAKE, FAKE, 16, 1.0, None, FAKE, FAKE, need, None) == ARG
     assert L.nvfp4_linear(FAKE, 4, 128, 1e-30, FAKE, FAKE, 16, 1e-30, None, FAKE, FAKE, need, None) == ARG
+    # the GEMM's own checks also run before the quantizer is launched (a
+    # launch here would fail with a CUDA error, not these codes)
+    assert L.nvfp4_linear(FAKE, 4, 128, 1.0, FAKE, FAKE, 16, 1.0, None, None, FAKE, need, None) == ARG     # Y
+    assert L.nvfp4_linear(FAKE, 4, 128, 1.0, FAKE + 4, FAKE, 16, 1.0, None, FAKE, FAKE, need, None) == ALIGN
+    assert L.nvfp4_linear(FAKE, 4, 128, 1.0, FAKE, FAKE, 12, 1.0, None, FAKE, FAKE, need, None) == SHAPE   # N % 8
+    assert L.nvfp4_linear(FAKE, 4, 128, 1e30, FAKE, FAKE, 16, 1e30, None, FAKE, FAKE, need, None) == ARG   # alpha -> 0
 
 
 def test_product_fails_loudly_without_library(tmp_path, monkeypatch):
