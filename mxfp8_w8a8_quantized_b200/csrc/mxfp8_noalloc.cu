@@ -60,8 +60,12 @@ extern "C" mxfp8_status mxfp8_linear_noalloc(const void *X, int64_t M, int64_t K
         return MXFP8_OK;
     if (!X || !Wq || !Wscale || !Y)
         return MXFP8_ERR_ARG;
-    if (K % 128 != 0)
+    if (K % 128 != 0 || N % 8 != 0)
         return MXFP8_ERR_SHAPE;
+    /* the GEMM's checks too, before the quantizer is launched */
+    const auto a16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+    if (!a16(X) || !a16(Wq) || !a16(Wscale) || !a16(Y) || (bias && !a16(bias)))
+        return MXFP8_ERR_ALIGN;
     /* the activation codes and their scales must fit the fixed scratch */
     if (M > MXFP8_NOALLOC_MAX_CODE_BYTES / K ||
         mxfp8_scale_bytes(M, K, MXFP8_SF_TCGEN05) > (size_t)MXFP8_NOALLOC_MAX_SCALE_BYTES)

@@ -216,3 +216,16 @@ def test_selftest_argument_checks(lib):
     assert lib.mxfp8_selftest_wait_timeout(-1, 1000000, None) == ARG
     assert lib.mxfp8_selftest_wait_timeout(0, 0, None) == ARG                # no limit
     assert lib.mxfp8_selftest_wait_timeout(0, 20_000_000_000, None) == ARG   # above 10 s
+
+
+def test_noalloc_rejects_before_launch(lib):
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    lib.mxfp8_linear_noalloc.argtypes = [P, I64, I64, P, P, I64, P, P, P]
+    ARG, ALIGN, SHAPE = 1, 2, 3
+    L = lib
+    assert L.mxfp8_linear_noalloc(FAKE, 4, 128, FAKE, FAKE, 12, None, FAKE, None) == SHAPE      # N % 8
+    assert L.mxfp8_linear_noalloc(FAKE, 4, 96, FAKE, FAKE, 16, None, FAKE, None) == SHAPE       # K % 128
+    assert L.mxfp8_linear_noalloc(FAKE, 4, 128, FAKE + 4, FAKE, 16, None, FAKE, None) == ALIGN  # Wq
+    assert L.mxfp8_linear_noalloc(FAKE, 4, 128, FAKE, FAKE, 16, FAKE + 2, FAKE, None) == ALIGN  # bias
+    assert L.mxfp8_linear_noalloc(FAKE, 4, 128, FAKE, FAKE, 16, None, None, None) == ARG        # Y
+    assert L.mxfp8_linear_noalloc(FAKE, 1 << 20, 5120, FAKE, FAKE, 16, None, FAKE, None) == SHAPE  # scratch
