@@ -51,7 +51,10 @@
  * per-row global stores.  Scale columns in TMEM are per stage, so a scale
  * copy never overwrites scales an earlier, still running MMA reads.  Every wait is bounded: on
  * timeout the kernel records MXFP8_ERR_TIMEOUT in a device status word,
- * drains its own MMAs, frees TMEM and returns.
+ * drains its own MMAs, lets copies still in flight land (a bounded settle),
+ * frees TMEM and returns.  Without block scales (the per-channel FP8 mode)
+ * TMEM holds two accumulators and the MMAs of the next tile overlap the
+ * epilogue of the last.
  */
 #include <cuda.h>
 #include <cuda_bf16.h>

@@ -45,7 +45,8 @@
  *                next tile into the other accumulator) and write Y through
  *                swizzled smem boxes and TMA stores.
  * Every wait is bounded: on timeout the kernel records the timeout in a
- * device status word, drains its own MMAs, frees TMEM and returns.
+ * device status word, drains its own MMAs, lets copies still in flight land
+ * (a bounded settle), frees TMEM and returns.
  */
 #include <cuda.h>
 #include <cuda_bf16.h>
