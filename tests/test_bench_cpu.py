@@ -124,3 +124,24 @@ def test_nvfp4_accounting():
     assert wl.tc_over_bf16 == 1.0 and wl.profile_kernel == "nvfp4_gemm"
     with pytest.raises(ValueError):
         bench.make_workload("c2_ffn_pair_832x1104", scheme="nvfp4")
+
+
+def test_traffic_is_reported_only_for_the_profiled_kernel_files(tmp_path, monkeypatch):
+    """roofline.traffic comes from profiles/<kernel>_<key>.json only while its
+    hash equals the hash of that kernel's current source files."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from mxfp8_w8a8_quantized_b200 import build
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    for kernel in ("mxfp8_gemm", "nvfp4_gemm"):
+        (prof / f"{kernel}_k.json").write_text(json.dumps(
+            {"kernel_source_sha": build.source_sha(kernel), "dram_bytes_per_launch": 123}))
+        assert bench.load_traffic("k", kernel) == 123
+        (prof / f"{kernel}_k.json").write_text(json.dumps(
+            {"kernel_source_sha": "0" * 16, "dram_bytes_per_launch": 123}))
+        assert bench.load_traffic("k", kernel) is None
+    assert bench.load_traffic("missing", "mxfp8_gemm") is None
+    # the two kernels hash different file sets; the library hash covers both
+    assert build.source_sha("mxfp8_gemm") != build.source_sha("nvfp4_gemm") != build.source_sha()
