@@ -107,7 +107,17 @@ def _stream():
 
 
 def _ptr(t):
-    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+    """Device address of a CUDA tensor of the current device (None -> NULL).
+    Every tensor handed to the library passes here, so host tensors and
+    tensors of another device are refused before a kernel could be given
+    their addresses."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError("tensor arguments must be CUDA tensors")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"tensor on {t.device}, but the current device is cuda:{torch.cuda.current_device()}")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _cuda(t, name, dtype=None):

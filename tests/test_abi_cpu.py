@@ -229,3 +229,35 @@ def test_noalloc_rejects_before_launch(lib):
     assert L.mxfp8_linear_noalloc(FAKE, 4, 128, FAKE, FAKE, 16, FAKE + 2, FAKE, None) == ALIGN  # bias
     assert L.mxfp8_linear_noalloc(FAKE, 4, 128, FAKE, FAKE, 16, None, None, None) == ARG        # Y
     assert L.mxfp8_linear_noalloc(FAKE, 1 << 20, 5120, FAKE, FAKE, 16, None, FAKE, None) == SHAPE  # scratch
+
+
+def test_binding_refuses_host_tensors():
+    """A host tensor never reaches the library: every wrapper raises
+    ValueError before the C call (a kernel given a host address would
+    fault)."""
+    import torch
+    from mxfp8_w8a8_quantized_b200 import mxfp8 as mx
+    u8 = lambda *s: torch.zeros(*s, dtype=torch.uint8)
+    f32 = lambda *s: torch.zeros(*s, dtype=torch.float32)
+    bf = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)
+    calls = [
+        lambda: mx.quantize(bf(4, 128)),
+        lambda: mx.quantize_weight(f32(8, 128)),
+        lambda: mx.linear(bf(4, 128), u8(8, 128), u8(512)),
+        lambda: mx.linear_noalloc(bf(4, 128), u8(8, 128), u8(512)),
+        lambda: mx.gemm_prequant(u8(4, 128), u8(512), u8(8, 128), u8(512)),
+        lambda: mx.gemm_quantize_out(u8(4, 128), u8(512), u8(128, 128), u8(512)),
+        lambda: mx.gelu_tanh(bf(64)),
+        lambda: mx.fp8rw_quantize(bf(4, 128)),
+        lambda: mx.fp8rw_quantize_weight(f32(8, 128)),
+        lambda: mx.fp8rw_gemm(u8(4, 128), f32(4), u8(8, 128), f32(8)),
+        lambda: mx.fp8rw_linear(bf(4, 128), u8(8, 128), f32(8)),
+        lambda: mx.nvfp4_amax(bf(64)),
+        lambda: mx.nvfp4_quantize(bf(4, 128), 1.0),
+        lambda: mx.nvfp4_quantize_weight(f32(8, 128), 1.0),
+        lambda: mx.nvfp4_gemm(u8(4, 64), u8(1024), u8(8, 64), u8(1024), 1.0),
+        lambda: mx.nvfp4_linear(bf(4, 128), 1.0, u8(8, 64), u8(1024), 1.0),
+    ]
+    for i, call in enumerate(calls):
+        with pytest.raises(ValueError):
+            call()
