@@ -823,26 +823,37 @@ def chain_oracle_sample(wl):
     return make
 
 
+def is_single_linear(wl):
+    return type(wl) in (LinearWorkload, FP8RowwiseLinearWorkload, NVFP4LinearWorkload)
+
+
+def size_chain(wl, target_s):
+    """A chained workload's oracle pass on a row sample grown until one pass
+    takes about target_s: (rows, run, flops of one pass, seconds of the last
+    sizing pass, description)."""
+    make = chain_oracle_sample(wl)
+    rows = 2
+    for _ in range(8):
+        run, fl = make(rows)
+        t0 = time.perf_counter()
+        run()
+        dt = time.perf_counter() - t0
+        if dt >= 0.5 * target_s or rows >= wl.M:
+            break
+        rows = int(min(wl.M, max(rows * 2, rows * 0.9 * target_s / max(dt, 1e-3))))
+    what = "the FFN pair" if isinstance(wl, FFNPairWorkload) else "one block (text linears on a proportional " \
+        "number of text rows)"
+    desc = f"{rows} video-token rows through {what}: quantize + FP64 linear per linear, GELU; weights quantized " \
+           "outside the timed region"
+    return rows, run, fl, dt, desc
+
+
 def cpu_baseline(wl, target_s):
     import oracle
-    if type(wl) not in (LinearWorkload, FP8RowwiseLinearWorkload, NVFP4LinearWorkload):
-        # chained: grow the row sample until one pass takes about target_s
-        make = chain_oracle_sample(wl)
-        rows = 2
-        for _ in range(8):
-            run, fl = make(rows)
-            t0 = time.perf_counter()
-            run()
-            dt = time.perf_counter() - t0
-            if dt >= 0.5 * target_s or rows >= wl.M:
-                break
-            rows = int(min(wl.M, max(rows * 2, rows * 0.9 * target_s / max(dt, 1e-3))))
-        what = "the FFN pair" if isinstance(wl, FFNPairWorkload) else "one block (text linears on a proportional " \
-            "number of text rows)"
+    if not is_single_linear(wl):
+        rows, run, fl, dt, desc = size_chain(wl, target_s)
         return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
-                "kind": "oracle",
-                "sample": f"{rows} video-token rows through {what}: quantize + FP64 linear per linear, GELU; "
-                          f"weights quantized outside the timed region; {dt:.1f} s"}
+                "kind": "oracle", "sample": f"{desc}; {dt:.1f} s"}
     rows = size_sample(wl, target_s)
     sample = oracle_sample(wl, rows)
     t0 = time.perf_counter()
@@ -858,22 +869,25 @@ def run_reference(args, ranks):
     """The oracle as the reference arm: CPU, rank 0 only."""
     import oracle
     wl = make_workload(args.workload, scheme=args.scheme)
-    if type(wl) not in (LinearWorkload, FP8RowwiseLinearWorkload, NVFP4LinearWorkload):
-        wl = LinearWorkload(wl.name, wl.M, wl.K, wl.K, wl.seed, wl.desc + " (first linear only)")
     if ranks.rank != 0:
         return None
     budget = args.reference_seconds  # warm-up + timed steps together
     n_steps = args.steps + args.warmup
-    rows = size_sample(wl, budget / n_steps)
-    sample = oracle_sample(wl, rows)
+    if is_single_linear(wl):
+        rows = size_sample(wl, budget / n_steps)
+        data = oracle_sample(wl, rows)
+        run, fl = (lambda: oracle_step(*data)), 2.0 * rows * wl.N * wl.K
+        sample = f"{rows} of {wl.M} rows per step (quantize + FP64 linear over all {wl.N} columns, K={wl.K})"
+    else:
+        rows, run, fl, _, desc = size_chain(wl, budget / n_steps)
+        sample = f"{desc}, per step"
     for _ in range(args.warmup):
-        oracle_step(*sample)
+        run()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(*sample)
+        run()
     dt = time.perf_counter() - t0
-    value = 2.0 * rows * wl.N * wl.K * args.steps / dt / 1e12
-    sample = f"{rows} of {wl.M} rows per step (quantize + FP64 linear over all {wl.N} columns, K={wl.K})"
+    value = fl * args.steps / dt / 1e12
     return {
         "impl": "reference",
         "metric": METRIC,

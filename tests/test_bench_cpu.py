@@ -145,3 +145,14 @@ def test_traffic_is_reported_only_for_the_profiled_kernel_files(tmp_path, monkey
     assert bench.load_traffic("missing", "mxfp8_gemm") is None
     # the two kernels hash different file sets; the library hash covers both
     assert build.source_sha("mxfp8_gemm") != build.source_sha("nvfp4_gemm") != build.source_sha()
+
+
+def test_reference_arm_times_the_whole_chain():
+    """For a chained workload the reference arm runs the oracle's chain
+    (both FFN linears and the GELU), the workload the GPU arm times."""
+    r = _bench(["--impl", "reference", "--workload", "c2_ffn_pair_832x1104", "--steps", "1", "--warmup", "1",
+                "--reference-seconds", "4"], {})
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads(r.stdout.strip().splitlines()[-1])
+    assert d["config"]["workload"] == "c2_ffn_pair_832x1104" and d["value"] > 0
+    assert "FFN pair" in d["cpu_baseline"]["sample"]
