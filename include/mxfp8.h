@@ -200,7 +200,9 @@ mxfp8_status mxfp8_gemm_quantize_out(const void *Xq, const void *Xscale, int64_t
  *   the library keeps until the process exits.
  *   First call on a device: looks up the scratch's device address
  *   (cudaGetSymbolAddress, with that device current) and caches it; make that
- *   first call before any stream capture.
+ *   first call before any stream capture.  cudaDeviceReset invalidates the
+ *   cached address: after resetting a device, do not call this entry point
+ *   on it again in the same process.
  *   Concurrency: all calls on a device share the one scratch array, which
  *   keeps the last call's contents.  Calls whose work overlaps on the GPU
  *   (different streams, or different host threads without ordering) race on

@@ -15,9 +15,14 @@
  * (34 MiB): every GPU that loads the library holds it until the process
  * exits.  Host code cannot use the variable's name as a device address, so
  * the first call on each device asks the runtime for its address
- * (cudaGetSymbolAddress, with that device current) and caches it.
+ * (cudaGetSymbolAddress, with that device current) and caches it.  The
+ * cache entries are atomics, so first calls from several host threads at
+ * once are well defined (each stores the same address).  A cudaDeviceReset
+ * destroys the context the address belongs to: a process that resets a
+ * device must not call mxfp8_linear_noalloc on it afterwards.
  */
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstdint>
 
 #include "mxfp8.h"
@@ -26,7 +31,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[MXFP8_NOALLOC_S
 
 namespace {
 
-void *g_scratch_addr[64] = {nullptr};
+std::atomic<void *> g_scratch_addr[64];
 
 /* Device address of the scratch array on the current device. */
 cudaError_t scratch_address(void **out)
@@ -37,14 +42,14 @@ cudaError_t scratch_address(void **out)
         return e;
     if (dev < 0 || dev >= 64)
         return cudaErrorInvalidDevice;
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
+    void *p = g_scratch_addr[dev].load(std::memory_order_relaxed);
+    if (!p) {
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess)
             return e;
-        g_scratch_addr[dev] = p;
+        g_scratch_addr[dev].store(p, std::memory_order_relaxed);
     }
-    *out = g_scratch_addr[dev];
+    *out = p;
     return cudaSuccess;
 }
 
