@@ -47,20 +47,23 @@ def rel_row_error(y: np.ndarray, yref: np.ndarray) -> np.ndarray:
     return num / np.maximum(den, 1e-300)
 
 
-# Drift allowed between the GPU chain and the exact chain, on top of twice the
-# drift between two admissible oracle evaluations (FP64 vs FP32 in k order).
+# Default band (the reduced-width block of tests/test_workloads_gpu.py): the
+# GPU chain's drift from the exact chain within twice the drift between two
+# admissible oracle evaluations (FP64 vs FP32 in k order), plus fixed slacks.
+CHAIN_FACTOR = 2.0
 CHAIN_MEAN_SLACK = 2e-3
 CHAIN_MAX_SLACK = 3e-2
 
 
-def chain_band(got, ref64, ref32):
+def chain_band(got, ref64, ref32, factor=CHAIN_FACTOR, mean_slack=CHAIN_MEAN_SLACK, max_slack=CHAIN_MAX_SLACK):
     """(ok, stats): the GPU chain's per-row relative drift from the exact
-    chain against the reference drift of the FP32-in-order oracle chain."""
+    chain against the reference drift of the FP32-in-order oracle chain:
+    mean D_gpu <= factor mean D_ref + mean_slack, and the same for the max."""
     d_gpu = rel_row_error(got, ref64)
     d_ref = rel_row_error(ref32, ref64)
     stats = dict(rows=len(got), gpu_mean=float(d_gpu.mean()), gpu_max=float(d_gpu.max()),
                  ref_mean=float(d_ref.mean()), ref_max=float(d_ref.max()))
     ok = (np.isfinite(got).all()
-          and d_gpu.mean() <= 2 * d_ref.mean() + CHAIN_MEAN_SLACK
-          and d_gpu.max() <= 2 * d_ref.max() + CHAIN_MAX_SLACK)
+          and d_gpu.mean() <= factor * d_ref.mean() + mean_slack
+          and d_gpu.max() <= factor * d_ref.max() + max_slack)
     return ok, stats

@@ -4,16 +4,25 @@
   at 832x1104; the first linears of a block): codes and scales bit-exact
   against the oracle, Y within |Y - Yref| <= 2^-7 |Yref| + 1e-3 rms(Yref) on
   sampled rows x columns (the ragged last tile and tile edges included).
-* Chains (FFN pair, one block, a 40-block step): every linear's BF16 output is
+* The FFN pair (ffn.net.0.proj -> GELU -> ffn.net.2, the model card's
+  "Coverage per transformer" dataflow): the chained output, element by
+  element on every sampled row (ragged tail included) and all 5120 columns,
+  within the same tolerance of the pure oracle chain -- FP64 linear, BF16,
+  the oracle's GELU, the oracle's quantization, FP64 linear.  Two linears
+  deep, the chain is not chaotic: a BF16 output that rounds the other way
+  moves at most a few re-quantized codes by one E4M3 step, far inside the
+  tolerance.
+* Deeper chains (one block, a 40-block step): every linear's BF16 output is
   one of several correct roundings (the FP32 accumulation order is not
   fixed), and a later linear re-quantizes it, so any two admissible
-  evaluations of a chain drift apart.  The exact oracle chain (FP64 sums) is
+  evaluations of a chain drift apart, and over six or more linears the
+  random-weight chain decorrelates.  The exact oracle chain (FP64 sums) is
   the reference; a second admissible evaluation -- the oracle with FP32
-  accumulation in increasing k -- gives the drift two valid evaluations
-  show on the same rows (D_ref).  The GPU chain's drift from the exact chain
-  (D_gpu, per-row relative L2) must stay within that band:
-      mean D_gpu <= 2 mean D_ref + 2e-3
-      max  D_gpu <= 2 max  D_ref + 3e-2     (oracle_chain.chain_band)
+  accumulation in increasing k -- gives the drift two valid evaluations show
+  on the same rows (D_ref).  The GPU chain's drift from the exact chain
+  (D_gpu, per-row relative L2) must stay within a band scaled to it:
+      mean D_gpu <= 1.5 mean D_ref + 1e-4
+      max  D_gpu <= 1.5 max  D_ref + 1e-4   (oracle_chain.chain_band)
 """
 import json
 import os
@@ -23,14 +32,19 @@ import pytest
 import torch
 
 import oracle
-from helpers import assert_within_tol, bf16_bits, bf16_values, f16_bits, unswizzle
+from helpers import assert_within_tol, bf16_bits, bf16_values, f16_bits, tol_violations, unswizzle
 from mxfp8_w8a8_quantized_b200 import synth
-from oracle_chain import OracleLinear, block_rows, chain_band
+from oracle_chain import OracleLinear, block_rows, chain_band, rel_row_error
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
+# Band of the deep chains (one block, 40 blocks): within 1.5x the drift of a
+# second admissible oracle evaluation, plus 1e-4 for the sampling of rows.
+DEEP_FACTOR, DEEP_SLACK = 1.5, 1e-4
+
+
 def check_chain(name, got, ref64, ref32):
-    ok, stats = chain_band(got, ref64, ref32)
+    ok, stats = chain_band(got, ref64, ref32, factor=DEEP_FACTOR, mean_slack=DEEP_SLACK, max_slack=DEEP_SLACK)
     record(name, **stats)
     assert ok, (name, stats)
 
@@ -142,19 +156,28 @@ def test_ffn_pair_832x1104_full_size(mx):
     del h
     torch.cuda.empty_cache()
 
-    # the chain: f -> GELU (in place) -> ffn.net.2
+    # the chain: f -> GELU (in place) -> ffn.net.2, element by element on all
+    # sampled rows and every column against the pure oracle chain
     wq2, ws2 = mx.quantize_weight(w2)
     mx.gelu_tanh(f, out=f)
     y = mx.linear(f, wq2, ws2, b2)
     torch.cuda.synchronize()
-    crow = rows[:: max(1, len(rows) // 24)]
-    x_rows = bf16_bits(x[torch.from_numpy(crow).to(DEV)])
+    assert mx.device_status() == 0
+    x_rows = bf16_bits(x[torch.from_numpy(rows).to(DEV)])
     lin0 = OracleLinear(w0.cpu().numpy(), f16_bits(b0))
     lin2 = OracleLinear(w2.cpu().numpy(), f16_bits(b2))
-    ref64 = bf16_values(lin2(oracle.gelu_tanh_bf16(lin0(x_rows))))
+    g_rows = oracle.gelu_tanh_bf16(lin0(x_rows))
+    yref = lin2.exact(g_rows)
+    got = bf16_values(bf16_bits(y[torch.from_numpy(rows).to(DEV)]))
+    assert got.shape == yref.shape == (len(rows), H)
+    bad, _ = tol_violations(got, yref)
     ref32 = bf16_values(lin2(oracle.gelu_tanh_bf16(lin0(x_rows, True)), True))
-    got = bf16_values(bf16_bits(y[torch.from_numpy(crow).to(DEV)]))
-    check_chain("ffn_pair_chain", got, ref64, ref32)
+    d_gpu = rel_row_error(got, yref)
+    d_ref = rel_row_error(ref32, yref)
+    record("ffn_pair_chain_elementwise", rows=len(rows), cols=H, outside=int(bad.sum()),
+           gpu_mean=float(d_gpu.mean()), gpu_max=float(d_gpu.max()),
+           ref_mean=float(d_ref.mean()), ref_max=float(d_ref.max()))
+    assert_within_tol(got, yref, "FFN pair chain")
 
 
 def test_ffn0_fused_epilogue_832x1104_full_size(mx):
