@@ -318,10 +318,10 @@ class FP8RowwiseLinearWorkload(LinearWorkload):
 class NVFP4LinearWorkload(LinearWorkload):
     """One NVFP4 linear: E2M1 codes with a UE4M3 scale per 16 elements and
     an FP32 global scale per tensor; Y = BF16(alpha (Xh . Wh^T) + b) with
-    alpha = 1 / (g_x g_w).  The weights' global scale comes from their amax
-    and the activations' from the amax of this workload's input, both
-    before timing (the activation scale is a calibrated constant of the
-    layer, not computed per step)."""
+    alpha = 1 / (g_x g_w), formed by the GEMM.  The weights' global scale
+    comes from their amax and the activations' from the amax of this
+    workload's input, both on the device before timing (the activation
+    scale is a calibrated constant of the layer, not computed per step)."""
 
     scheme = "nvfp4"
     gemm_kernel = "nvfp4_gemm_kernel"
@@ -349,9 +349,8 @@ class NVFP4LinearWorkload(LinearWorkload):
         self.x = synth.activations_device(M, K, s, 0, dev)
         w = synth.weights_device(N, K, s, 0, dev)
         self.b = synth.bias_device(N, s, 0, dev)
-        self.gw = mxfp8.nvfp4_global_scale(mxfp8.nvfp4_amax(w).item())
-        self.gx = mxfp8.nvfp4_global_scale(mxfp8.nvfp4_amax(self.x).item())
-        self.alpha = mxfp8.nvfp4_alpha(self.gx, self.gw)
+        self.gw = mxfp8.nvfp4_global_scale(w)           # device tensors; the GEMM forms alpha
+        self.gx = mxfp8.nvfp4_global_scale(self.x)
         self.wq, self.ws = mxfp8.nvfp4_quantize_weight(w, self.gw)   # offline weight quantization
         del w
         self.xq = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
@@ -362,7 +361,7 @@ class NVFP4LinearWorkload(LinearWorkload):
     def step(self, T):
         mx = self.mx
         T("quant", mx.nvfp4_quantize, self.x, self.gx, codes=self.xq, scales=self.xs)
-        T("gemm", mx.nvfp4_gemm, self.xq, self.xs, self.wq, self.ws, self.alpha, self.b, out=self.y)
+        T("gemm", mx.nvfp4_gemm, self.xq, self.xs, self.wq, self.ws, self.gx, self.gw, self.b, out=self.y)
 
     def e2e_step(self, x_dev, y_dev, ws):
         self.mx.nvfp4_linear(x_dev, self.gx, self.wq, self.ws, self.gw, self.b, out=y_dev, workspace=ws)

@@ -16,16 +16,17 @@ cudaError_t launch_gelu(const void *X, void *Y, int64_t n, cudaStream_t stream);
 int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void *Wq, const void *Ws, int64_t N,
                 const void *bias, void *Y, int epi, void *S, cudaStream_t stream, unsigned long long timeout_ns,
                 cudaError_t *err);
-cudaError_t launch_nvfp4_quantize(const void *X, bool f32_in, int64_t M, int64_t K, int64_t ldx, float g,
+cudaError_t launch_nvfp4_quantize(const void *X, bool f32_in, int64_t M, int64_t K, int64_t ldx, const float *g,
                                   uint8_t *Q, uint8_t *S, cudaStream_t stream);
 cudaError_t launch_nvfp4_amax(const void *X, bool f32_in, int64_t n, unsigned int *out, cudaStream_t stream);
+cudaError_t launch_nvfp4_global_scale(const float *amax, float *g, cudaStream_t stream);
 cudaError_t read_and_clear_status(unsigned int *out);
 cudaError_t launch_fp8_rowwise_quantize(const void *X, bool f32_in, int64_t M, int64_t K, int64_t ldx, uint8_t *Q,
                                         float *S, cudaStream_t stream, unsigned long long timeout_ns);
 cudaError_t read_and_clear_rw_status(unsigned int *out);
 int launch_nvfp4_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void *Wq, const void *Ws,
-                      int64_t N, float alpha, const void *bias, void *Y, cudaStream_t stream,
-                      unsigned long long timeout_ns, cudaError_t *err);
+                      int64_t N, const float *gx, const float *gw, const void *bias, void *Y,
+                      cudaStream_t stream, unsigned long long timeout_ns, cudaError_t *err);
 cudaError_t read_and_clear_nv_status(unsigned int *out);
 cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t stream);
 cudaError_t launch_nv_wait_selftest(unsigned long long limit_ns, cudaStream_t stream);
@@ -345,62 +346,73 @@ mxfp8_status nvfp4_amax_f32(const float *W, int64_t n, float *amax, mxfp8_stream
     return nvfp4_amax_any(W, true, n, amax, stream);
 }
 
-static mxfp8_status nvfp4_quantize_any(const void *X, bool f32, int64_t M, int64_t K, int64_t ldx, float g,
+mxfp8_status nvfp4_global_scale_from_amax(const float *amax, float *global_scale, mxfp8_stream_t stream)
+{
+    if (!amax || !global_scale)
+        return MXFP8_ERR_ARG;
+    if (!aligned(amax, 4) || !aligned(global_scale, 4))
+        return MXFP8_ERR_ALIGN;
+    return from_cuda(mx::launch_nvfp4_global_scale(amax, global_scale, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static mxfp8_status nvfp4_quantize_any(const void *X, bool f32, int64_t M, int64_t K, int64_t ldx, const float *g,
                                        void *codes, void *scales, mxfp8_stream_t stream)
 {
-    if (M < 0 || K <= 0 || ldx < K || !(g > 0.0f) || !(g < 3.0e38f))
+    if (M < 0 || K <= 0 || ldx < K)
         return MXFP8_ERR_ARG;
     if (M == 0)
         return MXFP8_OK;
-    if (!X || !codes || !scales)
+    if (!X || !g || !codes || !scales)
         return MXFP8_ERR_ARG;
     if (K % 16 != 0 || M > kMaxRows || K > kMaxK)
         return MXFP8_ERR_SHAPE;
-    if (!aligned(X, 16) || (ldx * (f32 ? 4 : 2)) % 16 != 0 || !aligned(codes, 8) || !aligned(scales, 4))
+    if (!aligned(X, 16) || (ldx * (f32 ? 4 : 2)) % 16 != 0 || !aligned(codes, 8) || !aligned(scales, 4) ||
+        !aligned(g, 4))
         return MXFP8_ERR_ALIGN;
     return from_cuda(mx::launch_nvfp4_quantize(X, f32, M, K, ldx, g, static_cast<uint8_t *>(codes),
                                                static_cast<uint8_t *>(scales),
                                                reinterpret_cast<cudaStream_t>(stream)));
 }
 
-mxfp8_status nvfp4_quantize_bf16(const void *X, int64_t M, int64_t K, int64_t ldx, float global_scale, void *codes,
-                                 void *scales, mxfp8_stream_t stream)
+mxfp8_status nvfp4_quantize_bf16(const void *X, int64_t M, int64_t K, int64_t ldx, const float *global_scale,
+                                 void *codes, void *scales, mxfp8_stream_t stream)
 {
     return nvfp4_quantize_any(X, false, M, K, ldx, global_scale, codes, scales, stream);
 }
 
-mxfp8_status nvfp4_quantize_weight_f32(const float *W, int64_t N, int64_t K, float global_scale, void *Wq,
+mxfp8_status nvfp4_quantize_weight_f32(const float *W, int64_t N, int64_t K, const float *global_scale, void *Wq,
                                        void *Wscale, mxfp8_stream_t stream)
 {
     return nvfp4_quantize_any(W, true, N, K, K, global_scale, Wq, Wscale, stream);
 }
 
 static mxfp8_status nvfp4_gemm_args(const void *Xq, const void *Xscale, int64_t M, int64_t K, const void *Wq,
-                                    const void *Wscale, int64_t N, float alpha, const void *bias, const void *Y)
+                                    const void *Wscale, int64_t N, const float *gx, const float *gw,
+                                    const void *bias, const void *Y)
 {
-    if (M < 0 || K <= 0 || N <= 0 || !(alpha > 0.0f) || !(alpha < 3.0e38f))
+    if (M < 0 || K <= 0 || N <= 0)
         return MXFP8_ERR_ARG;
     if (M == 0)
         return MXFP8_OK;
-    if (!Xq || !Xscale || !Wq || !Wscale || !Y)
+    if (!Xq || !Xscale || !Wq || !Wscale || !Y || !gx || !gw)
         return MXFP8_ERR_ARG;
     if (K % 64 != 0 || N % 8 != 0 || M > kMaxRows || N > kMaxRows || K > kMaxK)
         return MXFP8_ERR_SHAPE;
     if (!aligned(Xq, 16) || !aligned(Xscale, 16) || !aligned(Wq, 16) || !aligned(Wscale, 16) || !aligned(Y, 16) ||
-        (bias && !aligned(bias, 16)))
+        (bias && !aligned(bias, 16)) || !aligned(gx, 4) || !aligned(gw, 4))
         return MXFP8_ERR_ALIGN;
     return MXFP8_OK;
 }
 
 mxfp8_status nvfp4_gemm(const void *Xq, const void *Xscale, int64_t M, int64_t K, const void *Wq,
-                        const void *Wscale, int64_t N, float alpha, const void *bias, void *Y,
-                        mxfp8_stream_t stream)
+                        const void *Wscale, int64_t N, const float *x_global_scale, const float *w_global_scale,
+                        const void *bias, void *Y, mxfp8_stream_t stream)
 {
-    mxfp8_status st = nvfp4_gemm_args(Xq, Xscale, M, K, Wq, Wscale, N, alpha, bias, Y);
+    mxfp8_status st = nvfp4_gemm_args(Xq, Xscale, M, K, Wq, Wscale, N, x_global_scale, w_global_scale, bias, Y);
     if (st != MXFP8_OK || M == 0)
         return st;
     cudaError_t e;
-    int r = mx::launch_nvfp4_gemm(Xq, Xscale, M, K, Wq, Wscale, N, alpha, bias, Y,
+    int r = mx::launch_nvfp4_gemm(Xq, Xscale, M, K, Wq, Wscale, N, x_global_scale, w_global_scale, bias, Y,
                                   reinterpret_cast<cudaStream_t>(stream), kWaitLimitNs, &e);
     if (r == 1)
         return MXFP8_ERR_CUDA;
@@ -414,16 +426,15 @@ size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t K)
     return round_up((size_t)M * (size_t)(K / 2), 256) + nvfp4_scale_bytes(M, K);
 }
 
-mxfp8_status nvfp4_linear(const void *X, int64_t M, int64_t K, float x_global_scale, const void *Wq,
-                          const void *Wscale, int64_t N, float w_global_scale, const void *bias, void *Y,
+mxfp8_status nvfp4_linear(const void *X, int64_t M, int64_t K, const float *x_global_scale, const void *Wq,
+                          const void *Wscale, int64_t N, const float *w_global_scale, const void *bias, void *Y,
                           void *workspace, size_t ws_bytes, mxfp8_stream_t stream)
 {
-    if (M < 0 || K <= 0 || N <= 0 || !(x_global_scale > 0.0f) || !(w_global_scale > 0.0f) ||
-        !(x_global_scale < 3.0e38f) || !(w_global_scale < 3.0e38f))
+    if (M < 0 || K <= 0 || N <= 0)
         return MXFP8_ERR_ARG;
     if (M == 0)
         return MXFP8_OK;
-    if (!X || !workspace)
+    if (!X || !workspace || !x_global_scale)
         return MXFP8_ERR_ARG;
     if (K % 64 != 0)
         return MXFP8_ERR_SHAPE;
@@ -431,17 +442,17 @@ mxfp8_status nvfp4_linear(const void *X, int64_t M, int64_t K, float x_global_sc
         return MXFP8_ERR_ALIGN;
     if (ws_bytes < nvfp4_linear_workspace_bytes(M, K))
         return MXFP8_ERR_ARG;
-    const float alpha = (float)(1.0 / ((double)x_global_scale * (double)w_global_scale));
     uint8_t *codes = static_cast<uint8_t *>(workspace);
     uint8_t *scales = codes + round_up((size_t)M * (size_t)(K / 2), 256);
     /* every check of both steps before anything is launched */
-    mxfp8_status st = nvfp4_gemm_args(codes, scales, M, K, Wq, Wscale, N, alpha, bias, Y);
+    mxfp8_status st =
+        nvfp4_gemm_args(codes, scales, M, K, Wq, Wscale, N, x_global_scale, w_global_scale, bias, Y);
     if (st != MXFP8_OK)
         return st;
     st = nvfp4_quantize_bf16(X, M, K, K, x_global_scale, codes, scales, stream);
     if (st != MXFP8_OK)
         return st;
-    return nvfp4_gemm(codes, scales, M, K, Wq, Wscale, N, alpha, bias, Y, stream);
+    return nvfp4_gemm(codes, scales, M, K, Wq, Wscale, N, x_global_scale, w_global_scale, bias, Y, stream);
 }
 
 mxfp8_status mxfp8_selftest_wait_timeout(int which, uint64_t timeout_ns, mxfp8_stream_t stream)

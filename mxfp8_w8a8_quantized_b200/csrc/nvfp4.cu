@@ -76,7 +76,8 @@ __device__ __forceinline__ uint32_t nq_e2m1x8(float x0, float x1, float x2, floa
  */
 template <bool F32_IN>
 __global__ void __launch_bounds__(NQ_THREADS) nvfp4_quantize_kernel(const void *__restrict__ X, int64_t M, int64_t K,
-                                                                    int64_t ldx, float g, uint8_t *__restrict__ Q,
+                                                                    int64_t ldx, const float *__restrict__ gptr,
+                                                                    uint8_t *__restrict__ Q,
                                                                     uint8_t *__restrict__ S, int64_t Mrows,
                                                                     int64_t nseg, int64_t kg)
 {
@@ -85,6 +86,7 @@ __global__ void __launch_bounds__(NQ_THREADS) nvfp4_quantize_kernel(const void *
     const int64_t nwarps = ((int64_t)gridDim.x * NQ_THREADS) >> 5;
     const int64_t units = Mrows * nseg;
     const int nblocks = (int)(K >> 4);
+    const float g = __ldg(gptr);
     const float gs = __fdiv_rn(g, 6.0f);
     const int64_t stride = nwarps * NQ_UNROLL;
     const int nseg32 = (int)nseg;
@@ -181,6 +183,21 @@ __global__ void __launch_bounds__(256) nvfp4_amax_kernel(const void *__restrict_
         atomicMax(out, m);
 }
 
+/* The global scale g = RN(448 * 6 / amax) of a tensor whose amax is
+ * *amax_bits; 1 when amax is 0 (or not finite) or the quotient overflows,
+ * since then no finite scale maps the tensor onto the format's range. */
+__global__ void nvfp4_global_scale_kernel(const unsigned int *__restrict__ amax_bits, float *__restrict__ g)
+{
+    const float amax = __uint_as_float(*amax_bits);
+    float v = 1.0f;
+    if (amax > 0.0f && amax <= 3.4028235e38f) {
+        const float q = __fdiv_rn(448.0f * 6.0f, amax);
+        if (q <= 3.4028235e38f)
+            v = q;
+    }
+    *g = v;
+}
+
 static int nq_num_sms()
 {
     static int sms[64] = {0};
@@ -196,7 +213,7 @@ static int nq_num_sms()
     return sms[dev];
 }
 
-cudaError_t launch_nvfp4_quantize(const void *X, bool f32_in, int64_t M, int64_t K, int64_t ldx, float g,
+cudaError_t launch_nvfp4_quantize(const void *X, bool f32_in, int64_t M, int64_t K, int64_t ldx, const float *g,
                                   uint8_t *Q, uint8_t *S, cudaStream_t stream)
 {
     const int64_t Mrows = ((M + 127) / 128) * 128;
@@ -233,6 +250,12 @@ cudaError_t launch_nvfp4_amax(const void *X, bool f32_in, int64_t n, unsigned in
         nvfp4_amax_kernel<true><<<(unsigned)blocks, 256, 0, stream>>>(X, n16, out);
     else
         nvfp4_amax_kernel<false><<<(unsigned)blocks, 256, 0, stream>>>(X, n16, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_nvfp4_global_scale(const float *amax, float *g, cudaStream_t stream)
+{
+    nvfp4_global_scale_kernel<<<1, 1, 0, stream>>>(reinterpret_cast<const unsigned int *>(amax), g);
     return cudaGetLastError();
 }
 

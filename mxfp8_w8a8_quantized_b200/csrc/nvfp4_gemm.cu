@@ -108,7 +108,8 @@ struct Params {
     const uint8_t *sfa;  /* activation scales, tensor-core layout of 16-element blocks */
     const uint8_t *sfb;  /* weight scales, same layout */
     const __half *bias;  /* [N] or null */
-    float alpha;
+    const float *gx;     /* activation global scale (device) */
+    const float *gw;     /* weight global scale (device) */
     int M, N, K;
     int kg;              /* K / 64: scale atoms per 128 rows */
     int num_m, num_n, raster;
@@ -281,9 +282,9 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32_sync(uint32_t taddr, uint32_t
 
 /* Y = BF16(alpha acc + bias) for 32 rows x 32 columns, staged through a
  * 64-byte-swizzled smem box and written by one TMA store of the warp. */
-__device__ __forceinline__ void epilogue_piece(const uint32_t (&acc)[32], const Params &p, const CUtensorMap *tmap_y,
-                                               int row0, int colc, int lane, uint32_t buf, uint32_t rowbase,
-                                               uint32_t swz)
+__device__ __forceinline__ void epilogue_piece(const uint32_t (&acc)[32], const Params &p, float alpha,
+                                               const CUtensorMap *tmap_y, int row0, int colc, int lane,
+                                               uint32_t buf, uint32_t rowbase, uint32_t swz)
 {
     if (row0 >= p.M || colc >= p.N) /* whole box outside Y */
         return;
@@ -308,8 +309,8 @@ __device__ __forceinline__ void epilogue_piece(const uint32_t (&acc)[32], const 
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int a = 8 * j8 + 2 * j;
-            __nv_bfloat162 v = __floats2bfloat162_rn(fmaf(p.alpha, __uint_as_float(acc[a]), b[2 * j]),
-                                                     fmaf(p.alpha, __uint_as_float(acc[a + 1]), b[2 * j + 1]));
+            __nv_bfloat162 v = __floats2bfloat162_rn(fmaf(alpha, __uint_as_float(acc[a]), b[2 * j]),
+                                                     fmaf(alpha, __uint_as_float(acc[a + 1]), b[2 * j + 1]));
             o[j] = *reinterpret_cast<uint32_t *>(&v);
         }
         st_shared_v4(rowbase + ((((uint32_t)j8) ^ swz) << 4), o[0], o[1], o[2], o[3]);
@@ -479,6 +480,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t rowbase = buf + (uint32_t)lane * 64u;
         const uint32_t swz = ((uint32_t)lane >> 1) & 3u;
 
+        /* alpha = 1 / (g_x g_w): the product of two binary32 values is exact
+         * in FP64, the quotient is rounded to FP64 and then once to binary32 */
+        const float alpha = (float)(1.0 / ((double)__ldg(p.gx) * (double)__ldg(p.gw)));
         uint32_t it = 0, ir = 0, tl = 0;
         bool ok = true;
         bool pending = false;
@@ -506,7 +510,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     if (lane == 0)
                         mbar_arrive_cluster(mapa_shared(bar_tempty + 8 * ab, 0u));
                 }
-                epilogue_piece(acc, p, &tmap_y, row0, col0 + 32 * c, lane, buf, rowbase, swz);
+                epilogue_piece(acc, p, alpha, &tmap_y, row0, col0 + 32 * c, lane, buf, rowbase, swz);
             }
             ++tl;
             return true;
@@ -682,8 +686,8 @@ namespace mx {
  * Returns 0 ok, 1 tensor-map failure, 2 CUDA error (in *err).
  */
 int launch_nvfp4_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void *Wq, const void *Ws,
-                      int64_t N, float alpha, const void *bias, void *Y, cudaStream_t stream,
-                      unsigned long long timeout_ns, cudaError_t *err)
+                      int64_t N, const float *gx, const float *gw, const void *bias, void *Y,
+                      cudaStream_t stream, unsigned long long timeout_ns, cudaError_t *err)
 {
     *err = cudaSuccess;
     if (M == 0)
@@ -703,7 +707,8 @@ int launch_nvfp4_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, cons
     p.sfa = static_cast<const uint8_t *>(Xs);
     p.sfb = static_cast<const uint8_t *>(Ws);
     p.bias = static_cast<const __half *>(bias);
-    p.alpha = alpha;
+    p.gx = gx;
+    p.gw = gw;
     p.M = (int)M;
     p.N = (int)N;
     p.K = (int)K;

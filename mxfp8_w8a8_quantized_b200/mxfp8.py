@@ -54,22 +54,23 @@ _lib.fp8rw_linear_workspace_bytes.argtypes = [_I64, _I64]
 _lib.fp8rw_linear_workspace_bytes.restype = _SZ
 _lib.fp8rw_linear.argtypes = [_P, _I64, _I64, _P, _P, _I64, _P, _P, _P, _SZ, _P]
 _lib.fp8rw_linear.restype = ctypes.c_int
-_F = ctypes.c_float
 _lib.nvfp4_scale_bytes.argtypes = [_I64, _I64]
 _lib.nvfp4_scale_bytes.restype = _SZ
 _lib.nvfp4_amax_bf16.argtypes = [_P, _I64, _P, _P]
 _lib.nvfp4_amax_bf16.restype = ctypes.c_int
 _lib.nvfp4_amax_f32.argtypes = [_P, _I64, _P, _P]
 _lib.nvfp4_amax_f32.restype = ctypes.c_int
-_lib.nvfp4_quantize_bf16.argtypes = [_P, _I64, _I64, _I64, _F, _P, _P, _P]
+_lib.nvfp4_global_scale_from_amax.argtypes = [_P, _P, _P]
+_lib.nvfp4_global_scale_from_amax.restype = ctypes.c_int
+_lib.nvfp4_quantize_bf16.argtypes = [_P, _I64, _I64, _I64, _P, _P, _P, _P]
 _lib.nvfp4_quantize_bf16.restype = ctypes.c_int
-_lib.nvfp4_quantize_weight_f32.argtypes = [_P, _I64, _I64, _F, _P, _P, _P]
+_lib.nvfp4_quantize_weight_f32.argtypes = [_P, _I64, _I64, _P, _P, _P, _P]
 _lib.nvfp4_quantize_weight_f32.restype = ctypes.c_int
-_lib.nvfp4_gemm.argtypes = [_P, _P, _I64, _I64, _P, _P, _I64, _F, _P, _P, _P]
+_lib.nvfp4_gemm.argtypes = [_P, _P, _I64, _I64, _P, _P, _I64, _P, _P, _P, _P, _P]
 _lib.nvfp4_gemm.restype = ctypes.c_int
 _lib.nvfp4_linear_workspace_bytes.argtypes = [_I64, _I64]
 _lib.nvfp4_linear_workspace_bytes.restype = _SZ
-_lib.nvfp4_linear.argtypes = [_P, _I64, _I64, _F, _P, _P, _I64, _F, _P, _P, _P, _SZ, _P]
+_lib.nvfp4_linear.argtypes = [_P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _P, _P, _SZ, _P]
 _lib.nvfp4_linear.restype = ctypes.c_int
 _lib.mxfp8_selftest_wait_timeout.argtypes = [ctypes.c_int, ctypes.c_uint64, _P]
 _lib.mxfp8_selftest_wait_timeout.restype = ctypes.c_int
@@ -87,7 +88,8 @@ EXPORTS = ("mxfp8_status_str", "mxfp8_scale_bytes", "mxfp8_quantize", "mxfp8_qua
            "mxfp8_gemm_quantize_out", "mxfp8_selftest_wait_timeout",
            "fp8rw_quantize_bf16", "fp8rw_quantize_weight_f32", "fp8rw_gemm", "fp8rw_linear_workspace_bytes",
            "fp8rw_linear",
-           "nvfp4_scale_bytes", "nvfp4_amax_bf16", "nvfp4_amax_f32", "nvfp4_quantize_bf16",
+           "nvfp4_scale_bytes", "nvfp4_amax_bf16", "nvfp4_amax_f32", "nvfp4_global_scale_from_amax",
+           "nvfp4_quantize_bf16",
            "nvfp4_quantize_weight_f32", "nvfp4_gemm", "nvfp4_linear_workspace_bytes", "nvfp4_linear")
 
 
@@ -309,17 +311,29 @@ def nvfp4_amax(t: torch.Tensor) -> torch.Tensor:
     return out
 
 
-def nvfp4_global_scale(amax: float) -> float:
-    """448 * 6 / amax in binary32 (the tensor's largest block gets the
-    largest UE4M3 scale)."""
-    import numpy as np
-    return float(np.float32(np.float32(448.0 * 6.0) / np.float32(amax)))
+def nvfp4_global_scale(t: torch.Tensor) -> torch.Tensor:
+    """The tensor's global scale RN(448 * 6 / amax) (1 for an all-zero
+    tensor), computed on the device: a 1-element FP32 CUDA tensor."""
+    amax = nvfp4_amax(t)
+    g = torch.empty(1, dtype=torch.float32, device=t.device)
+    _check(_lib.nvfp4_global_scale_from_amax(_ptr(amax), _ptr(g), _stream()), "nvfp4_global_scale_from_amax")
+    return g
 
 
-def nvfp4_quantize(x: torch.Tensor, global_scale: float, codes=None, scales=None):
-    """BF16 [M, K] -> (packed E2M1 codes uint8 [M, K/2], UE4M3 scales, tensor-core layout)."""
+def _scale_tensor(g: torch.Tensor, what: str):
+    if not isinstance(g, torch.Tensor):
+        raise ValueError(f"{what} must be a 1-element FP32 CUDA tensor")
+    _cuda(g, what, torch.float32)
+    if g.numel() != 1:
+        raise ValueError(f"{what} must hold one FP32 value (a global scale)")
+
+
+def nvfp4_quantize(x: torch.Tensor, global_scale: torch.Tensor, codes=None, scales=None):
+    """BF16 [M, K] -> (packed E2M1 codes uint8 [M, K/2], UE4M3 scales, tensor-core
+    layout) with the global scale held in a 1-element FP32 CUDA tensor."""
     if not x.is_cuda or x.dtype != torch.bfloat16 or x.dim() != 2:
         raise ValueError("x must be a 2-D BF16 CUDA tensor")
+    _scale_tensor(global_scale, "global_scale")
     M, K = x.shape
     ldx = x.stride(0) if M > 1 else K
     if x.stride(1) != 1 or ldx < K:
@@ -328,37 +342,36 @@ def nvfp4_quantize(x: torch.Tensor, global_scale: float, codes=None, scales=None
         codes = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
     if scales is None:
         scales = torch.empty(max(nvfp4_scale_bytes(M, K), 1), dtype=torch.uint8, device=x.device)
-    _check(_lib.nvfp4_quantize_bf16(_ptr(x), M, K, ldx, global_scale, _ptr(codes), _ptr(scales), _stream()),
-           "nvfp4_quantize_bf16")
+    _check(_lib.nvfp4_quantize_bf16(_ptr(x), M, K, ldx, _ptr(global_scale), _ptr(codes), _ptr(scales),
+                                    _stream()), "nvfp4_quantize_bf16")
     return codes, scales
 
 
-def nvfp4_quantize_weight(w: torch.Tensor, global_scale: float):
+def nvfp4_quantize_weight(w: torch.Tensor, global_scale: torch.Tensor):
     """FP32 [N, K] (rounded to BF16 first) -> (packed codes [N, K/2], scales)."""
     _cuda(w, "w", torch.float32)
+    _scale_tensor(global_scale, "global_scale")
     N, K = w.shape
     codes = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device)
     scales = torch.empty(max(nvfp4_scale_bytes(N, K), 1), dtype=torch.uint8, device=w.device)
-    _check(_lib.nvfp4_quantize_weight_f32(_ptr(w), N, K, global_scale, _ptr(codes), _ptr(scales), _stream()),
-           "nvfp4_quantize_weight_f32")
+    _check(_lib.nvfp4_quantize_weight_f32(_ptr(w), N, K, _ptr(global_scale), _ptr(codes), _ptr(scales),
+                                          _stream()), "nvfp4_quantize_weight_f32")
     return codes, scales
 
 
-def nvfp4_alpha(x_global_scale: float, w_global_scale: float) -> float:
-    """alpha = 1 / (g_x g_w), rounded once to binary32 (as nvfp4_linear)."""
-    import numpy as np
-    return float(np.float32(1.0 / (float(x_global_scale) * float(w_global_scale))))
-
-
-def nvfp4_gemm(xq, xscale, wq, wscale, alpha: float, bias=None, out=None):
+def nvfp4_gemm(xq, xscale, wq, wscale, x_global_scale: torch.Tensor, w_global_scale: torch.Tensor, bias=None,
+               out=None):
     """Y = BF16(alpha sum_k (qx dec(sx)) (qw dec(sw)) + bias) from NVFP4
-    operands: packed codes [M, K/2] / [N, K/2] and their scales."""
+    operands: packed codes [M, K/2] / [N, K/2], their scales, and the two
+    global scales (1-element FP32 CUDA tensors; the kernel forms alpha)."""
+    _scale_tensor(x_global_scale, "x_global_scale")
+    _scale_tensor(w_global_scale, "w_global_scale")
     M, K2 = xq.shape
     N = wq.shape[0]
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
-    _check(_lib.nvfp4_gemm(_ptr(xq), _ptr(xscale), M, 2 * K2, _ptr(wq), _ptr(wscale), N, alpha, _ptr(bias),
-                           _ptr(out), _stream()), "nvfp4_gemm")
+    _check(_lib.nvfp4_gemm(_ptr(xq), _ptr(xscale), M, 2 * K2, _ptr(wq), _ptr(wscale), N, _ptr(x_global_scale),
+                           _ptr(w_global_scale), _ptr(bias), _ptr(out), _stream()), "nvfp4_gemm")
     return out
 
 
@@ -366,19 +379,20 @@ def nvfp4_linear_workspace_bytes(M: int, K: int) -> int:
     return int(_lib.nvfp4_linear_workspace_bytes(M, K))
 
 
-def nvfp4_linear(x: torch.Tensor, x_global_scale: float, wq, wscale, w_global_scale: float, bias=None, out=None,
-                 workspace=None):
-    """The NVFP4 layer: quantize x with its global scale, then nvfp4_gemm
-    with alpha = 1 / (g_x g_w)."""
+def nvfp4_linear(x: torch.Tensor, x_global_scale: torch.Tensor, wq, wscale, w_global_scale: torch.Tensor, bias=None,
+                 out=None, workspace=None):
+    """The NVFP4 layer: quantize x with its global scale, then nvfp4_gemm."""
     _cuda(x, "x", torch.bfloat16)
+    _scale_tensor(x_global_scale, "x_global_scale")
+    _scale_tensor(w_global_scale, "w_global_scale")
     M, K = x.shape
     N = wq.shape[0]
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     if workspace is None:
         workspace = torch.empty(max(nvfp4_linear_workspace_bytes(M, K), 256), dtype=torch.uint8, device=x.device)
-    _check(_lib.nvfp4_linear(_ptr(x), M, K, x_global_scale, _ptr(wq), _ptr(wscale), N, w_global_scale, _ptr(bias),
-                             _ptr(out), _ptr(workspace), workspace.numel(), _stream()), "nvfp4_linear")
+    _check(_lib.nvfp4_linear(_ptr(x), M, K, _ptr(x_global_scale), _ptr(wq), _ptr(wscale), N, _ptr(w_global_scale),
+                             _ptr(bias), _ptr(out), _ptr(workspace), workspace.numel(), _stream()), "nvfp4_linear")
     return out
 
 

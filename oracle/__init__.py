@@ -316,6 +316,14 @@ def nvfp4_linear(xq, xs, gx, wq, ws, gw, bias_bits=None, rows=None, cols=None):
 
 
 def nvfp4_global_scale(amax):
-    """The per-tensor global scale 448 * 6 / amax (binary32): the largest
-    block then gets the largest UE4M3 scale."""
-    return np.float32(np.float32(448.0 * 6.0) / np.float32(amax))
+    """The per-tensor global scale 448 * 6 / amax (binary32 division): the
+    largest block then gets the largest UE4M3 scale.  When amax is 0 or not
+    finite, or the quotient overflows, no finite scale maps the tensor onto
+    the format's range and the scale is 1 (reading: the page gives the field,
+    not its value for an all-zero tensor)."""
+    a = np.float32(amax)
+    if not (a > 0 and np.isfinite(a)):
+        return np.float32(1.0)
+    with np.errstate(over="ignore"):
+        q = np.float32(np.float32(448.0 * 6.0) / a)
+    return q if np.isfinite(q) else np.float32(1.0)

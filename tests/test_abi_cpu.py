@@ -149,34 +149,41 @@ def test_fp8_rowwise_argument_checks_return_before_launch(lib):
 
 
 def test_nvfp4_gemm_argument_checks_return_before_launch(lib):
-    P, I64, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float
-    lib.nvfp4_gemm.argtypes = [P, P, I64, I64, P, P, I64, F, P, P, P]
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    lib.nvfp4_gemm.argtypes = [P, P, I64, I64, P, P, I64, P, P, P, P, P]
     lib.nvfp4_linear_workspace_bytes.argtypes = [I64, I64]
     lib.nvfp4_linear_workspace_bytes.restype = ctypes.c_size_t
-    lib.nvfp4_linear.argtypes = [P, I64, I64, F, P, P, I64, F, P, P, P, ctypes.c_size_t, P]
+    lib.nvfp4_linear.argtypes = [P, I64, I64, P, P, P, I64, P, P, P, P, ctypes.c_size_t, P]
+    lib.nvfp4_global_scale_from_amax.argtypes = [P, P, P]
+    lib.nvfp4_quantize_bf16.argtypes = [P, I64, I64, I64, P, P, P, P]
     L = lib
     ARG, ALIGN, SHAPE = 1, 2, 3
-    assert L.nvfp4_gemm(FAKE, FAKE, 4, 96, FAKE, FAKE, 16, 1.0, None, FAKE, None) == SHAPE    # K % 64
-    assert L.nvfp4_gemm(FAKE, FAKE, 4, 128, FAKE, FAKE, 12, 1.0, None, FAKE, None) == SHAPE   # N % 8
-    assert L.nvfp4_gemm(FAKE, FAKE + 4, 4, 128, FAKE, FAKE, 16, 1.0, None, FAKE, None) == ALIGN
-    assert L.nvfp4_gemm(FAKE, FAKE, 4, 128, FAKE, FAKE, 16, 1.0, FAKE + 2, FAKE, None) == ALIGN  # bias
-    assert L.nvfp4_gemm(FAKE, FAKE, 4, 128, FAKE, FAKE, 16, 0.0, None, FAKE, None) == ARG     # alpha > 0
-    assert L.nvfp4_gemm(FAKE, FAKE, 4, 128, FAKE, FAKE, 16, float("inf"), None, FAKE, None) == ARG
-    assert L.nvfp4_gemm(FAKE, FAKE, 4, 128, FAKE, None, 16, 1.0, None, FAKE, None) == ARG
-    assert L.nvfp4_gemm(FAKE, FAKE, 0, 128, FAKE, FAKE, 16, 1.0, None, FAKE, None) == 0
+    G = FAKE                                     # a device float holding a global scale
+    assert L.nvfp4_gemm(FAKE, FAKE, 4, 96, FAKE, FAKE, 16, G, G, None, FAKE, None) == SHAPE    # K % 64
+    assert L.nvfp4_gemm(FAKE, FAKE, 4, 128, FAKE, FAKE, 12, G, G, None, FAKE, None) == SHAPE   # N % 8
+    assert L.nvfp4_gemm(FAKE, FAKE + 4, 4, 128, FAKE, FAKE, 16, G, G, None, FAKE, None) == ALIGN
+    assert L.nvfp4_gemm(FAKE, FAKE, 4, 128, FAKE, FAKE, 16, G, G, FAKE + 2, FAKE, None) == ALIGN  # bias
+    assert L.nvfp4_gemm(FAKE, FAKE, 4, 128, FAKE, FAKE, 16, None, G, None, FAKE, None) == ARG     # g_x
+    assert L.nvfp4_gemm(FAKE, FAKE, 4, 128, FAKE, FAKE, 16, G, None, None, FAKE, None) == ARG     # g_w
+    assert L.nvfp4_gemm(FAKE, FAKE, 4, 128, FAKE, FAKE, 16, G + 2, G, None, FAKE, None) == ALIGN  # float alignment
+    assert L.nvfp4_gemm(FAKE, FAKE, 4, 128, FAKE, None, 16, G, G, None, FAKE, None) == ARG
+    assert L.nvfp4_gemm(FAKE, FAKE, 0, 128, FAKE, FAKE, 16, G, G, None, FAKE, None) == 0
     need = L.nvfp4_linear_workspace_bytes(4, 128)
     assert need == 256 + 2 * 512                 # codes rounded to 256 B + one row block of 2 scale atoms
-    assert L.nvfp4_linear(FAKE, 4, 128, 1.0, FAKE, FAKE, 16, 1.0, None, FAKE, FAKE, need - 1, None) == ARG
-    assert L.nvfp4_linear(FAKE, 4, 128, 1.0, FAKE, FAKE, 16, 1.0, None, FAKE, FAKE + 16, need, None) == ALIGN
-    assert L.nvfp4_linear(FAKE, 4, 96, 1.0, FAKE, FAKE, 16, 1.0, None, FAKE, FAKE, need, None) == SHAPE
-    assert L.nvfp4_linear(FAKE, 4, 128, 0.0, FAKE, FAKE, 16, 1.0, None, FAKE, FAKE, need, None) == ARG
-    assert L.nvfp4_linear(FAKE, 4, 128, 1e-30, FAKE, FAKE, 16, 1e-30, None, FAKE, FAKE, need, None) == ARG
+    assert L.nvfp4_linear(FAKE, 4, 128, G, FAKE, FAKE, 16, G, None, FAKE, FAKE, need - 1, None) == ARG
+    assert L.nvfp4_linear(FAKE, 4, 128, G, FAKE, FAKE, 16, G, None, FAKE, FAKE + 16, need, None) == ALIGN
+    assert L.nvfp4_linear(FAKE, 4, 96, G, FAKE, FAKE, 16, G, None, FAKE, FAKE, need, None) == SHAPE
+    assert L.nvfp4_linear(FAKE, 4, 128, None, FAKE, FAKE, 16, G, None, FAKE, FAKE, need, None) == ARG
     # the GEMM's own checks also run before the quantizer is launched (a
     # launch here would fail with a CUDA error, not these codes)
-    assert L.nvfp4_linear(FAKE, 4, 128, 1.0, FAKE, FAKE, 16, 1.0, None, None, FAKE, need, None) == ARG     # Y
-    assert L.nvfp4_linear(FAKE, 4, 128, 1.0, FAKE + 4, FAKE, 16, 1.0, None, FAKE, FAKE, need, None) == ALIGN
-    assert L.nvfp4_linear(FAKE, 4, 128, 1.0, FAKE, FAKE, 12, 1.0, None, FAKE, FAKE, need, None) == SHAPE   # N % 8
-    assert L.nvfp4_linear(FAKE, 4, 128, 1e30, FAKE, FAKE, 16, 1e30, None, FAKE, FAKE, need, None) == ARG   # alpha -> 0
+    assert L.nvfp4_linear(FAKE, 4, 128, G, FAKE, FAKE, 16, None, None, FAKE, FAKE, need, None) == ARG    # g_w
+    assert L.nvfp4_linear(FAKE, 4, 128, G, FAKE, FAKE, 16, G, None, None, FAKE, need, None) == ARG       # Y
+    assert L.nvfp4_linear(FAKE, 4, 128, G, FAKE + 4, FAKE, 16, G, None, FAKE, FAKE, need, None) == ALIGN
+    assert L.nvfp4_linear(FAKE, 4, 128, G, FAKE, FAKE, 12, G, None, FAKE, FAKE, need, None) == SHAPE     # N % 8
+    assert L.nvfp4_global_scale_from_amax(None, G, None) == ARG
+    assert L.nvfp4_global_scale_from_amax(G, G + 1, None) == ALIGN
+    assert L.nvfp4_quantize_bf16(FAKE, 4, 128, 128, None, FAKE, FAKE, None) == ARG                      # g
+    assert L.nvfp4_quantize_bf16(FAKE, 4, 128, 128, G + 2, FAKE, FAKE, None) == ALIGN
 
 
 def test_product_fails_loudly_without_library(tmp_path, monkeypatch):
@@ -229,6 +236,9 @@ def test_noalloc_rejects_before_launch(lib):
     assert L.mxfp8_linear_noalloc(FAKE, 4, 128, FAKE, FAKE, 16, FAKE + 2, FAKE, None) == ALIGN  # bias
     assert L.mxfp8_linear_noalloc(FAKE, 4, 128, FAKE, FAKE, 16, None, None, None) == ARG        # Y
     assert L.mxfp8_linear_noalloc(FAKE, 1 << 20, 5120, FAKE, FAKE, 16, None, FAKE, None) == SHAPE  # scratch
+    assert L.mxfp8_linear_noalloc(FAKE, 6554, 5120, FAKE, FAKE, 16, None, FAKE, None) == SHAPE     # codes cap + 1 row
+    # codes fit (32 x 524416 B), the scales (4 x 524416 B > 2 MiB) do not
+    assert L.mxfp8_linear_noalloc(FAKE, 32, (1 << 19) + 128, FAKE, FAKE, 16, None, FAKE, None) == SHAPE
 
 
 def test_binding_refuses_host_tensors():
@@ -253,10 +263,11 @@ def test_binding_refuses_host_tensors():
         lambda: mx.fp8rw_gemm(u8(4, 128), f32(4), u8(8, 128), f32(8)),
         lambda: mx.fp8rw_linear(bf(4, 128), u8(8, 128), f32(8)),
         lambda: mx.nvfp4_amax(bf(64)),
-        lambda: mx.nvfp4_quantize(bf(4, 128), 1.0),
-        lambda: mx.nvfp4_quantize_weight(f32(8, 128), 1.0),
-        lambda: mx.nvfp4_gemm(u8(4, 64), u8(1024), u8(8, 64), u8(1024), 1.0),
-        lambda: mx.nvfp4_linear(bf(4, 128), 1.0, u8(8, 64), u8(1024), 1.0),
+        lambda: mx.nvfp4_global_scale(bf(64)),
+        lambda: mx.nvfp4_quantize(bf(4, 128), f32(1)),
+        lambda: mx.nvfp4_quantize_weight(f32(8, 128), f32(1)),
+        lambda: mx.nvfp4_gemm(u8(4, 64), u8(1024), u8(8, 64), u8(1024), f32(1), f32(1)),
+        lambda: mx.nvfp4_linear(bf(4, 128), f32(1), u8(8, 64), u8(1024), f32(1)),
     ]
     for i, call in enumerate(calls):
         with pytest.raises(ValueError):

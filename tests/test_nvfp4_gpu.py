@@ -1,6 +1,9 @@
-"""GPU parity of the NVFP4 quantizers against the CPU oracle: packed E2M1
-codes and UE4M3 scales bit-exact (both sides take the same binary32 steps),
-tensor amax exact."""
+"""GPU parity of the NVFP4 path against the CPU oracle: packed E2M1 codes
+and UE4M3 scales bit-exact (both sides take the same binary32 steps), the
+tensor amax and the global scale exact -- the GPU forms its global scale on
+the device, the oracle forms its own from the host copy of the same tensor,
+and the two must be the same binary32 value -- and the GEMM within the
+output tolerance."""
 import numpy as np
 import pytest
 import torch
@@ -19,18 +22,41 @@ def mx():
 
 
 def _g(mx, t):
-    amax = mx.nvfp4_amax(t).item()
-    return mx.nvfp4_global_scale(amax), amax
+    """(device global scale tensor, the oracle's global scale from the host
+    values, host amax).  The FP32 weights are measured after rounding to
+    BF16, as the weight quantizer sees them."""
+    host = bf16_values(bf16_bits(t.to(torch.bfloat16)))
+    amax = float(np.abs(host).max()) if host.size else 0.0
+    g_ref = oracle.nvfp4_global_scale(amax)
+    g_dev = mx.nvfp4_global_scale(t)
+    torch.cuda.synchronize()
+    assert mx.nvfp4_amax(t).item() == amax
+    assert g_dev.cpu().numpy().view(np.uint32)[0] == np.float32(g_ref).view(np.uint32), (g_dev.item(), g_ref)
+    return g_dev, g_ref
+
+
+def _dev(g):
+    """A global scale chosen by the test, as the 1-element device tensor the
+    library takes."""
+    return torch.tensor([g], dtype=torch.float32, device="cuda")
+
+
+def test_global_scale_on_device(mx):
+    """448 * 6 / amax in binary32 on the device, 1 for an all-zero tensor."""
+    for t, g in ((torch.zeros(64, dtype=torch.bfloat16), 1.0),
+                 (torch.full((32,), 2688.0, dtype=torch.bfloat16), 1.0),
+                 (torch.full((16,), -3.0, dtype=torch.bfloat16), 896.0)):
+        dg, rg = _g(mx, t.cuda())
+        assert float(rg) == g and dg.item() == g
 
 
 @pytest.mark.parametrize("M,K", [(256, 512), (1, 16), (300, 5120), (129, 13824), (1000, 1040), (64, 48)])
 def test_activation_quantizer_bit_exact(mx, M, K):
     x = synth.activations_device(M, K, M + K, 0, "cuda")
-    g, amax = _g(mx, x)
-    assert amax == float(np.abs(bf16_values(bf16_bits(x))).max())
+    g, g_ref = _g(mx, x)
     codes, scales = mx.nvfp4_quantize(x, g)
     torch.cuda.synchronize()
-    rq, rs = oracle.nvfp4_quantize_bf16(bf16_bits(x), g)
+    rq, rs = oracle.nvfp4_quantize_bf16(bf16_bits(x), g_ref)
     assert np.array_equal(codes.cpu().numpy(), rq)
     assert np.array_equal(unswizzle(scales.cpu().numpy(), M, K, 16), rs)
 
@@ -43,13 +69,13 @@ def test_activation_quantizer_edge_blocks_and_strides(mx):
     x[2, :16] = -0.0
     x[3, 16:32] = 1e-30                         # scale underflows to 0 -> codes +-0
     x[4, 5] = 3.0e4                             # one huge element
-    g = 448.0 * 6.0 / 3.0e4
-    codes, scales = mx.nvfp4_quantize(x, g)
+    g = float(np.float32(448.0 * 6.0 / 3.0e4))
+    codes, scales = mx.nvfp4_quantize(x, _dev(g))
     torch.cuda.synchronize()
     rq, rs = oracle.nvfp4_quantize_bf16(bf16_bits(x), g)
     assert np.array_equal(codes.cpu().numpy(), rq)
     assert np.array_equal(unswizzle(scales.cpu().numpy(), M, K, 16), rs)
-    c2, s2 = mx.nvfp4_quantize(x.contiguous(), g)
+    c2, s2 = mx.nvfp4_quantize(x.contiguous(), _dev(g))
     torch.cuda.synchronize()
     assert torch.equal(codes, c2) and torch.equal(scales, s2)
 
@@ -57,12 +83,11 @@ def test_activation_quantizer_edge_blocks_and_strides(mx):
 @pytest.mark.parametrize("N,K", [(512, 512), (333, 13824), (8, 16)])
 def test_weight_quantizer_rounds_to_bf16_first(mx, N, K):
     w = synth.weights_device(N, K, N + K, 0, "cuda")
-    g, amax = _g(mx, w)
+    g, g_ref = _g(mx, w)
     wb = bf16_bits(w.to(torch.bfloat16))
-    assert amax == float(np.abs(bf16_values(wb)).max())
     codes, scales = mx.nvfp4_quantize_weight(w, g)
     torch.cuda.synchronize()
-    rq, rs = oracle.nvfp4_quantize_bf16(wb, g)
+    rq, rs = oracle.nvfp4_quantize_bf16(wb, g_ref)
     assert np.array_equal(codes.cpu().numpy(), rq)
     assert np.array_equal(unswizzle(scales.cpu().numpy(), N, K, 16), rs)
 
@@ -76,13 +101,14 @@ def _nv_layer(mx, M, K, N, seed, with_bias=True):
     x = synth.activations_device(M, K, seed, 0, "cuda")
     w = synth.weights_device(N, K, seed, 0, "cuda")
     b = synth.bias_device(N, seed, 0, "cuda") if with_bias else None
-    gx, _ = _g(mx, x)
-    gw, _ = _g(mx, w)
+    gx, gx_ref = _g(mx, x)
+    gw, gw_ref = _g(mx, w)
     wq, ws = mx.nvfp4_quantize_weight(w, gw)
-    return x, w, b, gx, gw, wq, ws
+    return x, w, b, (gx, gx_ref), (gw, gw_ref), wq, ws
 
 
 def _oracle_y(x, w, b, gx, gw, rows=None, cols=None):
+    """The oracle's layer with its own (host) global scales."""
     rq, rs = oracle.nvfp4_quantize_bf16(bf16_bits(x), gx)
     oq, os_ = oracle.nvfp4_quantize_bf16(bf16_bits(w.to(torch.bfloat16)), gw)
     bb = None if b is None else b.cpu().view(torch.int16).numpy().view(np.uint16)
@@ -92,14 +118,14 @@ def _oracle_y(x, w, b, gx, gw, rows=None, cols=None):
 @pytest.mark.parametrize("M,K,N", [(256, 512, 512), (300, 512, 384), (1, 64, 8), (129, 256, 640),
                                    (1000, 1088, 1536), (517, 13824, 264), (260, 320, 520)])
 def test_gemm_within_tolerance(mx, M, K, N):
-    x, w, b, gx, gw, wq, ws = _nv_layer(mx, M, K, N, seed=M + N)
+    x, w, b, (gx, gx_ref), (gw, gw_ref), wq, ws = _nv_layer(mx, M, K, N, seed=M + N)
     xq, xs = mx.nvfp4_quantize(x, gx)
-    y = mx.nvfp4_gemm(xq, xs, wq, ws, mx.nvfp4_alpha(gx, gw), b)
+    y = mx.nvfp4_gemm(xq, xs, wq, ws, gx, gw, b)
     y2 = mx.nvfp4_linear(x, gx, wq, ws, gw, b)
     torch.cuda.synchronize()
     assert mx.device_status() == 0
     assert torch.equal(y, y2), "nvfp4_linear differs from quantize + gemm"
-    yref = _oracle_y(x, w, b, gx, gw)
+    yref = _oracle_y(x, w, b, gx_ref, gw_ref)
     assert_within_tol(bf16_values(bf16_bits(y)), yref, f"nvfp4 {M}x{K}x{N}")
 
 
@@ -120,9 +146,10 @@ def test_gemm_exact_grid_values(mx):
 
     xv, wv = make(M), make(N)
     x = xv.to(torch.bfloat16).cuda()
-    xq, xs = mx.nvfp4_quantize(x, 1.0)
-    wq, ws = mx.nvfp4_quantize_weight(wv.cuda(), 1.0)
-    y = mx.nvfp4_gemm(xq, xs, wq, ws, 1.0, None)
+    one = _dev(1.0)
+    xq, xs = mx.nvfp4_quantize(x, one)
+    wq, ws = mx.nvfp4_quantize_weight(wv.cuda(), one)
+    y = mx.nvfp4_gemm(xq, xs, wq, ws, one, one, None)
     torch.cuda.synchronize()
     assert np.all(unswizzle(xs.cpu().numpy(), M, K, 16) == 0x38)
     exact = xv.double().numpy() @ wv.double().numpy().T
@@ -132,31 +159,34 @@ def test_gemm_exact_grid_values(mx):
 def test_gemm_q_projection_480p_full_size_sampled(mx):
     """M = 32760, K = N = 5120: codes and scales bit-exact, sampled Y."""
     M, K, N, seed = synth.TOKENS_480P, synth.HIDDEN, synth.HIDDEN, 1
-    x, w, b, gx, gw, wq, ws = _nv_layer(mx, M, K, N, seed)
+    x, w, b, (gx, gx_ref), (gw, gw_ref), wq, ws = _nv_layer(mx, M, K, N, seed)
     xq, xs = mx.nvfp4_quantize(x, gx)
-    y = mx.nvfp4_gemm(xq, xs, wq, ws, mx.nvfp4_alpha(gx, gw), b)
+    y = mx.nvfp4_gemm(xq, xs, wq, ws, gx, gw, b)
     torch.cuda.synchronize()
     assert mx.device_status() == 0
-    rq, rs = oracle.nvfp4_quantize_bf16(bf16_bits(x), gx)
+    rq, rs = oracle.nvfp4_quantize_bf16(bf16_bits(x), gx_ref)
     assert np.array_equal(xq.cpu().numpy(), rq)
     assert np.array_equal(unswizzle(xs.cpu().numpy(), M, K, 16), rs)
-    oq, os_ = oracle.nvfp4_quantize_bf16(bf16_bits(w.to(torch.bfloat16)), gw)
+    oq, os_ = oracle.nvfp4_quantize_bf16(bf16_bits(w.to(torch.bfloat16)), gw_ref)
     rng = np.random.default_rng(0)
     rows = np.unique(np.concatenate([[0, 127, 128, 255, 256, M - 129, M - 1], np.arange(M - 40, M),
                                      rng.choice(M, 150, replace=False)]))
     cols = np.unique(np.concatenate([[0, 8, 255, 256, N - 1], rng.choice(N, 120, replace=False)]))
     bb = b.cpu().view(torch.int16).numpy().view(np.uint16)
-    yref = oracle.nvfp4_linear(rq, rs, gx, oq, os_, gw, bb, rows=rows, cols=cols)
+    yref = oracle.nvfp4_linear(rq, rs, gx_ref, oq, os_, gw_ref, bb, rows=rows, cols=cols)
     got = y[torch.from_numpy(rows).cuda()][:, torch.from_numpy(cols).cuda()]
     assert_within_tol(bf16_values(bf16_bits(got)), yref, "nvfp4 Q projection")
 
 
 def test_gemm_argument_errors(mx):
     x = torch.zeros((4, 96), dtype=torch.bfloat16, device="cuda")
-    xq, xs = mx.nvfp4_quantize(x, 1.0)
+    one = _dev(1.0)
+    xq, xs = mx.nvfp4_quantize(x, one)
     w = torch.zeros((8, 96), dtype=torch.float32, device="cuda")
-    wq, ws = mx.nvfp4_quantize_weight(w, 1.0)
+    wq, ws = mx.nvfp4_quantize_weight(w, one)
     with pytest.raises(mx.MXFP8Error):          # K = 96 is not a multiple of 64
-        mx.nvfp4_gemm(xq, xs, wq, ws, 1.0)
-    with pytest.raises(mx.MXFP8Error):          # alpha must be finite and > 0
-        mx.nvfp4_gemm(xq, xs, wq, ws, 0.0)
+        mx.nvfp4_gemm(xq, xs, wq, ws, one, one)
+    with pytest.raises(ValueError):             # a global scale is a 1-element FP32 CUDA tensor
+        mx.nvfp4_gemm(xq, xs, wq, ws, 1.0, one)
+    with pytest.raises(ValueError):
+        mx.nvfp4_quantize(x, torch.ones(2, device="cuda"))

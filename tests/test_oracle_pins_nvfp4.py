@@ -151,3 +151,18 @@ def test_zero_block_gets_zero_scale_and_signed_zero_codes():
     q, s = oracle.nvfp4_quantize_bf16(_bits(x), np.float32(448 * 6))
     assert s[0, 0] == 0 and np.all(q[0, :8] == 0x88)
     assert oracle.e4m3_decode(s[0, 1]) == 448
+
+
+def test_global_scale_landmarks():
+    """g = 448 * 6 / amax as a binary32 division (numpy's), which maps the
+    tensor's largest block scale to 448 (the UE4M3 maximum); an all-zero,
+    non-finite or underflowing amax gives 1."""
+    for a in (1.0, 3.0, 0.1, 2688.0, 1e-30, 8e-36):
+        want = np.float32(2688.0) / np.float32(a)
+        assert oracle.nvfp4_global_scale(a) == want
+        # the block holding amax gets the largest scale: amax g / 6 == 448
+        assert abs(float(np.float32(a) * want / np.float32(6.0)) / 448.0 - 1.0) < 1e-6
+    assert oracle.nvfp4_global_scale(0.0) == 1.0
+    assert oracle.nvfp4_global_scale(float("inf")) == 1.0
+    assert oracle.nvfp4_global_scale(float("nan")) == 1.0
+    assert oracle.nvfp4_global_scale(1e-38) == 1.0          # 2688 / 1e-38 overflows binary32
