@@ -5,11 +5,14 @@ One step = one pass of the whole hot path over one batch: dynamic MX
 quantization of every BF16 activation and the block-scaled tcgen05 GEMM
 with its F16-bias / BF16 epilogue for every linear of the workload (plus the
 GELU between the FFN linears).  Weights are quantized once, offline, before
-timing.  Default workload: the Wan2.2 A14B self-attention Q projection at
-480x832, 81 frames (M = 32760 tokens, K = N = 5120).
+timing.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME]
+
+Default workload: one denoising step of Wan2.2 A14B at 832x1104, 81 frames
+(40 blocks x 10 quantized linears, 75348 video / 512 text tokens), the
+largest single-GPU configuration and the one holding both FFN shapes.
 
 Prints ONE JSON line (rank 0).  `value` is whole-job TFLOP/s (2*M*N*K summed
 over the step's linears, over all GPUs, divided by the slowest rank's device
@@ -37,15 +40,15 @@ FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_BF16_SUSTAINED = 1400.0
 FP8_OVER_BF16 = 2.0  # nominal dense ratio: 4.5 PF/s FP8 vs 2.25 PF/s BF16
 L2_FLUSH_BYTES = 256 << 20
-WORKLOADS = ["c1_q_proj_480p", "c0_small", "ffn0_832x1104", "ffn2_832x1104",
-             "c2_ffn_pair_832x1104", "c3_block_832x1104", "c4_step_832x1104"]
+WORKLOADS = ["c4_step_832x1104", "c1_q_proj_480p", "c0_small", "ffn0_832x1104", "ffn2_832x1104",
+             "c2_ffn_pair_832x1104", "c3_block_832x1104"]
 
 
 def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOADS[0], choices=WORKLOADS)
     ap.add_argument("--unfused", action="store_true",
@@ -169,13 +172,20 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- timing
+def call_label(fn):
+    """The linear a call runs, when the callee is a named linear (or one of
+    its methods); None otherwise."""
+    return getattr(fn, "name", None) or getattr(getattr(fn, "__self__", None), "name", None)
+
+
 class KernelTimer:
     """CUDA events around each library call of a step, on the launching
-    stream: per-kind device time (GEMM, quantizer, GELU)."""
+    stream: per-kind device time (GEMM, quantizer, GELU), and per linear for
+    the GEMMs of named linears."""
 
     def __init__(self, stream):
         self.stream = stream
-        self.events = []          # (kind, start, end)
+        self.events = []          # (kind, label, start, end)
         self.on = False
 
     def __call__(self, kind, fn, *a, **kw):
@@ -185,14 +195,23 @@ class KernelTimer:
         s.record(self.stream)
         r = fn(*a, **kw)
         e.record(self.stream)
-        self.events.append((kind, s, e))
+        self.events.append((kind, call_label(fn), s, e))
         return r
 
     def totals(self):
         out = {}
-        for kind, s, e in self.events:
+        for kind, _, s, e in self.events:
             n, t = out.get(kind, (0, 0.0))
             out[kind] = (n + 1, t + s.elapsed_time(e))
+        return out
+
+    def per_label(self, kind="gemm"):
+        """{label: (launches, total ms)} over the calls of `kind` that carry a label."""
+        out = {}
+        for k, label, s, e in self.events:
+            if k == kind and label is not None:
+                n, t = out.get(label, (0, 0.0))
+                out[label] = (n + 1, t + s.elapsed_time(e))
         return out
 
 
@@ -217,6 +236,10 @@ class LinearWorkload:
 
     def config(self):
         return {"M": self.M, "K": self.K, "N": self.N}
+
+    def linear_flops(self):
+        """FLOPs of one launch of each named GEMM (none for a single linear)."""
+        return {}
 
     def flops(self):
         return 2.0 * self.M * self.N * self.K
@@ -389,6 +412,9 @@ class FFNPairWorkload(LinearWorkload):
     def flops(self):
         return 2 * 2.0 * self.M * self.N * self.K
 
+    def linear_flops(self):
+        return {"ffn.net.0.proj": 2.0 * self.M * self.K * self.N, "ffn.net.2": 2.0 * self.M * self.N * self.K}
+
     def quant_bytes(self):
         q = _quant_bytes(self.M, self.K)
         return q if self.fused else q + _quant_bytes(self.M, self.N)
@@ -405,6 +431,7 @@ class FFNPairWorkload(LinearWorkload):
         self.x = synth.activations_device(M, H, s, 0, dev)
         self.l0 = QLinear.random(H, F, s, 1, dev)
         self.l2 = QLinear.random(F, H, s, 2, dev)
+        self.l0.name, self.l2.name = "ffn.net.0.proj", "ffn.net.2"
         self.wsx = Workspace(M * H, M, H, dev)
         self.wsf = Workspace(M * F, M, F, dev)
         self.f = None if self.fused else torch.empty((M, F), dtype=torch.bfloat16, device=dev)
@@ -462,6 +489,18 @@ class BlocksWorkload(LinearWorkload):
             gemms = [(M if kind == "video" else T, K, N, False) for _, K, N, kind in synth.block_linears()]
             quants = [(M, H)] * 5 + [(T, H), (M, F)]
         return gemms, quants
+
+    def linear_flops(self):
+        """FLOPs of one launch of each named GEMM of a block."""
+        H, F, M, T = self.K, self.N, self.M, self.T
+        if self.fused:
+            out = {"attn1.to_qkv": 2.0 * M * H * 3 * H, "attn2.to_kv": 2.0 * T * H * 2 * H}
+        else:
+            out = {n: 2.0 * M * H * H for n in ("attn1.to_q", "attn1.to_k", "attn1.to_v")}
+            out.update({n: 2.0 * T * H * H for n in ("attn2.to_k", "attn2.to_v")})
+        out.update({"attn1.to_out": 2.0 * M * H * H, "attn2.to_q": 2.0 * M * H * H, "attn2.to_out": 2.0 * M * H * H,
+                    "ffn.net.0.proj": 2.0 * M * H * F, "ffn.net.2": 2.0 * M * F * H})
+        return out
 
     def _per_block(self):
         gemms, quants = self._launches()
@@ -541,6 +580,12 @@ def make_workload(name, fused=True, scheme="mxfp8"):
     raise ValueError(name)
 
 
+def run_config(wl, world):
+    """The `config` object of the JSON line; both arms print the same one."""
+    return dict(workload=wl.name, desc=wl.desc, **wl.config(),
+                parallelism=f"replicas x{world}" if world > 1 else "single GPU")
+
+
 # ---------------------------------------------------------------- our arm
 def run_ours(args, ranks, dev):
     wl = make_workload(args.workload, fused=not args.unfused, scheme=args.scheme)
@@ -617,10 +662,9 @@ def run_ours(args, ranks, dev):
         "dtype": wl.dtype,
         "data": "synthetic (seeded N(0,1) activations with 1% x20 outlier channels, N(0,1/sqrt(K)) weights, "
                 "N(0,0.01) f16 bias)",
-        "config": dict(workload=wl.name, desc=wl.desc, **wl.config(),
-                       l2="flushed between timed steps (256 MiB write outside the step events)",
-                       launch="one CUDA graph per step" if graph is not None else "eager launches",
-                       parallelism=f"replicas x{ranks.world}" if ranks.world > 1 else "single GPU"),
+        "config": run_config(wl, ranks.world),
+        "timing": {"l2": "flushed between timed steps (256 MiB write outside the step events)",
+                   "launch": "one CUDA graph per step" if graph is not None else "eager launches"},
         "roofline": {"bound": "tensor", "kernel": wl.gemm_kernel,
                      "achieved": round(gemm_tflops, 1), "peak": round(tc_peak, 1), "unit": "TFLOP/s",
                      "frac": round(gemm_tflops / tc_peak, 4),
@@ -637,6 +681,15 @@ def run_ours(args, ranks, dev):
         "gpu_launches": wl.launches * steps,
         "clocks": clk.summary(),
     }
+    lf = wl.linear_flops()
+    per = {}
+    for label, (n, ms) in sorted(T.per_label("gemm").items()):
+        if label in lf:
+            tf = lf[label] * n / (ms * 1e-3) / 1e12
+            per[label] = {"launches_per_step": n // kernel_steps, "avg_launch_ms": round(ms / n, 4),
+                          "achieved": round(tf, 1), "frac": round(tf / tc_peak, 4)}
+    if per:
+        out["roofline"]["per_linear"] = per
     if "gelu" in tot:
         n, ms = tot["gelu"]
         out["gelu"] = {"launches_per_step": n // kernel_steps, "avg_launch_ms": round(ms / n, 4)}
@@ -901,7 +954,7 @@ def run_reference(args, ranks):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (same recipe as the GPU arm)",
-        "config": dict(workload=wl.name, desc=wl.desc, **wl.config()),
+        "config": run_config(wl, ranks.world),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -39,10 +39,11 @@ BLOCK_LINEARS = [name for name, _, _, _ in synth.block_linears()]
 
 
 class QLinear:
-    """One quantized linear: MXFP8 weight codes + tensor-core scales, F16 bias."""
+    """One quantized linear: MXFP8 weight codes + tensor-core scales, F16 bias.
+    `name` labels it (the model card's module name) for per-linear timing."""
 
-    def __init__(self, wq, ws, bias, K, N):
-        self.wq, self.ws, self.bias, self.K, self.N = wq, ws, bias, K, N
+    def __init__(self, wq, ws, bias, K, N, name=None):
+        self.wq, self.ws, self.bias, self.K, self.N, self.name = wq, ws, bias, K, N, name
 
     @classmethod
     def concat(cls, parts):
@@ -108,6 +109,9 @@ class Block:
         self.qkv, (L["attn1.to_q"], L["attn1.to_k"], L["attn1.to_v"]) = QLinear.concat(
             [L["attn1.to_q"], L["attn1.to_k"], L["attn1.to_v"]])
         self.kv2, (L["attn2.to_k"], L["attn2.to_v"]) = QLinear.concat([L["attn2.to_k"], L["attn2.to_v"]])
+        for name, lin in L.items():
+            lin.name = name
+        self.qkv.name, self.kv2.name = "attn1.to_qkv", "attn2.to_kv"
 
     def forward(self, x, ctx, ws_a, ws_b, keep=False, fuse_qkv=True, fuse_ffn=True, timer=None):
         """x [M, hidden], ctx [T, hidden] BF16.  ws_a / ws_b: two Workspaces

@@ -103,6 +103,32 @@ def test_fused_accounting():
     assert bf.flops() == bp.flops()
 
 
+def test_per_linear_accounting_covers_the_step():
+    """Every GEMM of a block is one named linear; their FLOPs add up to the
+    workload's (so the per-linear rooflines cover the whole step), and the
+    default workload is the 40-block step."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.parse([]).workload == "c4_step_832x1104"
+    for fused in (True, False):
+        for name in ("c3_block_832x1104", "c4_step_832x1104", "c2_ffn_pair_832x1104"):
+            wl = bench.make_workload(name, fused=fused)
+            per_block = sum(wl.linear_flops().values())
+            blocks = getattr(wl, "nblocks", 1)
+            assert blocks * per_block == pytest.approx(wl.flops()), (name, fused)
+    assert bench.make_workload("c1_q_proj_480p").linear_flops() == {}
+
+
+def test_both_arms_print_the_same_config():
+    sys.path.insert(0, ROOT)
+    import bench
+    r = _bench(["--impl", "reference", "--workload", "c0_small", "--steps", "1", "--warmup", "1",
+                "--reference-seconds", "2"], {})
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["config"] == bench.run_config(bench.make_workload("c0_small"), 1)
+
+
 @pytest.mark.parametrize("scheme", ["fp8rowwise", "nvfp4"])
 def test_reference_arm_other_schemes(scheme):
     r = _bench(["--impl", "reference", "--workload", "c0_small", "--scheme", scheme, "--steps", "2",
