@@ -50,3 +50,11 @@ def assert_within_tol(y: np.ndarray, yref: np.ndarray, what=""):
         idx = np.argwhere(bad)[:5]
         det = [(tuple(i), float(y[tuple(i)]), float(yref[tuple(i)]), float(bound[tuple(i)])) for i in idx]
         raise AssertionError(f"{what}: {int(bad.sum())} of {bad.size} outside tolerance, e.g. {det}")
+
+
+def mx_values(codes: np.ndarray, scales_rowmajor: np.ndarray, block: int = 32) -> np.ndarray:
+    """Dequantized MXFP8 values (FP64) of E4M3 codes [rows, K] with E8M0
+    scales [rows, K/block], decoded with torch's float8_e4m3fn."""
+    c = torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    e = scales_rowmajor.astype(np.float64) - 127.0
+    return c * np.repeat(np.exp2(e), block, axis=1)

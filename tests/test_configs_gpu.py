@@ -5,13 +5,21 @@
   against the oracle, Y within |Y - Yref| <= 2^-7 |Yref| + 1e-3 rms(Yref) on
   sampled rows x columns (the ragged last tile and tile edges included).
 * The FFN pair (ffn.net.0.proj -> GELU -> ffn.net.2, the model card's
-  "Coverage per transformer" dataflow): the chained output, element by
-  element on every sampled row (ragged tail included) and all 5120 columns,
-  within the same tolerance of the pure oracle chain -- FP64 linear, BF16,
-  the oracle's GELU, the oracle's quantization, FP64 linear.  Two linears
-  deep, the chain is not chaotic: a BF16 output that rounds the other way
-  moves at most a few re-quantized codes by one E4M3 step, far inside the
-  tolerance.
+  "Coverage per transformer" dataflow), element by element on every sampled
+  row (ragged tail included) and all 5120 columns, against the pure oracle
+  chain (FP64 linear, BF16, the oracle's GELU and quantization, FP64
+  linear).  The BF16 values feeding ffn.net.2's quantization are admissible
+  roundings (FP32 sum order, GELU evaluation) that differ from the exact
+  chain's in a few places, and a value that rounds the other way can move
+  its E4M3 code by one step: about 5e-4 on an output, the size of the
+  1e-3 rms term.  So the bound is the stated tolerance of the last linear
+  plus the exact effect of those input differences:
+      |Y - Yref| <= 2^-7 (|Yref| + A) + 1e-3 (rms(Yref) + rms(A)) + A,
+      A[m, n] = sum_k |xq_gpu[m, k] - xq_ref[m, k]| |wq[n, k]|
+  (xq: dequantized ffn.net.2 inputs, the GPU's from its own quantizer, the
+  reference's from the oracle chain), with at most 1e-3 of the inputs
+  differing.  Rows whose inputs equal the oracle's get A = 0: the stated
+  tolerance exactly.
 * Deeper chains (one block, a 40-block step): every linear's BF16 output is
   one of several correct roundings (the FP32 accumulation order is not
   fixed), and a later linear re-quantizes it, so any two admissible
@@ -32,7 +40,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import assert_within_tol, bf16_bits, bf16_values, f16_bits, tol_violations, unswizzle
+from helpers import assert_within_tol, bf16_bits, bf16_values, f16_bits, mx_values, tol_violations, unswizzle
 from mxfp8_w8a8_quantized_b200 import synth
 from oracle_chain import OracleLinear, block_rows, chain_band, rel_row_error
 
@@ -161,23 +169,42 @@ def test_ffn_pair_832x1104_full_size(mx):
     wq2, ws2 = mx.quantize_weight(w2)
     mx.gelu_tanh(f, out=f)
     y = mx.linear(f, wq2, ws2, b2)
+    gq, gs = mx.quantize(f)                     # ffn.net.2's input as mxfp8_linear quantizes it
     torch.cuda.synchronize()
     assert mx.device_status() == 0
-    x_rows = bf16_bits(x[torch.from_numpy(rows).to(DEV)])
+    rows_t = torch.from_numpy(rows).to(DEV)
+    x_rows = bf16_bits(x[rows_t])
     lin0 = OracleLinear(w0.cpu().numpy(), f16_bits(b0))
     lin2 = OracleLinear(w2.cpu().numpy(), f16_bits(b2))
     g_rows = oracle.gelu_tanh_bf16(lin0(x_rows))
     yref = lin2.exact(g_rows)
-    got = bf16_values(bf16_bits(y[torch.from_numpy(rows).to(DEV)]))
+    got = bf16_values(bf16_bits(y[rows_t]))
     assert got.shape == yref.shape == (len(rows), H)
-    bad, _ = tol_violations(got, yref)
+    # the inputs of ffn.net.2: the GPU's against the oracle chain's
+    rq, rs = oracle.quantize_bf16(g_rows)
+    xq_ref = mx_values(rq, rs)
+    xq_gpu = mx_values(gq[rows_t].cpu().numpy(), unswizzle(gs.cpu().numpy(), M, F)[rows])
+    dx = np.abs(xq_gpu - xq_ref)
+    differing = float((dx > 0).mean())
+    assert differing <= 1e-3, f"{differing:.2e} of ffn.net.2's inputs differ from the oracle chain"
+    A = dx @ np.abs(mx_values(lin2.wq, lin2.ws)).T
+    rms = float(np.sqrt(np.mean(yref ** 2)))
+    # the last linear's tolerance around the exact output on the GPU's own
+    # input (which lies within A of Yref), plus A
+    bound = 2.0 ** -7 * (np.abs(yref) + A) + 1e-3 * (rms + float(np.sqrt(np.mean(A ** 2)))) + A
+    err = np.abs(got - yref)
+    clean = ~(dx > 0).any(axis=1)
     ref32 = bf16_values(lin2(oracle.gelu_tanh_bf16(lin0(x_rows, True)), True))
-    d_gpu = rel_row_error(got, yref)
-    d_ref = rel_row_error(ref32, yref)
-    record("ffn_pair_chain_elementwise", rows=len(rows), cols=H, outside=int(bad.sum()),
-           gpu_mean=float(d_gpu.mean()), gpu_max=float(d_gpu.max()),
-           ref_mean=float(d_ref.mean()), ref_max=float(d_ref.max()))
-    assert_within_tol(got, yref, "FFN pair chain")
+    d_gpu, d_ref = rel_row_error(got, yref), rel_row_error(ref32, yref)
+    plain_bad, _ = tol_violations(got, yref)
+    record("ffn_pair_chain_elementwise", rows=len(rows), cols=H, inputs_differing=differing,
+           rows_with_equal_inputs=int(clean.sum()), outside_stated_tol=int(plain_bad.sum()),
+           max_err_over_bound=float((err / bound).max()), gpu_mean=float(d_gpu.mean()),
+           gpu_max=float(d_gpu.max()), ref_mean=float(d_ref.mean()), ref_max=float(d_ref.max()))
+    assert np.isfinite(got).all()
+    bad = err > bound
+    assert not bad.any(), f"FFN pair chain: {int(bad.sum())} outputs outside the bound, worst " \
+                          f"{float((err / bound).max()):.3g} x"
 
 
 def test_ffn0_fused_epilogue_832x1104_full_size(mx):

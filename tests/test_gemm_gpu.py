@@ -46,6 +46,9 @@ def gpu_linear(mx, x, w, b):
     (129, 384, 264),     # ragged M and N tails
     (300, 128, 520),
     (513, 640, 1024),    # several tiles in both directions
+    (260, 256, 896),     # three and a half 256-wide tiles
+    (131, 384, 1160),    # four 256-wide tiles and a 136-column tail
+    (64, 128, 232),      # one partial tile
 ])
 def test_linear_vs_oracle(mx, M, K, N):
     seed = 0 if (M, K, N) == (256, 512, 512) else M + N
@@ -83,12 +86,13 @@ def test_exact_when_accumulation_is_exact(mx):
     assert np.array_equal(bf16_bits(y), oracle.bf16_rne(yref))
 
 
-def test_scale_placement_probe(mx):
+@pytest.mark.parametrize("N", [512, 1024])
+def test_scale_placement_probe(mx, N):
     # every code is 1.0; each (row, block) and (column, block) gets its own
     # scale, so a misplaced scale byte anywhere shows up as a wrong power of
-    # two in some output.
+    # two in some output (N = 1024: four tiles along N)
     rng = np.random.default_rng(9)
-    M, K, N = 256, 512, 512
+    M, K = 256, 512
     nb = K // 32
     ex = rng.integers(-2, 3, (M, nb))
     ew = rng.integers(-2, 3, (N, nb))
