@@ -78,7 +78,9 @@ constexpr uint32_t ACC_COL = 0; /* 256 FP32 columns */
 /* M tiles walked together (for every N tile) so that their A rows stay in
  * L2: 8 when the weights fit in L2 alongside them, 16 when the weights are
  * re-read from DRAM once per group (measured: ffn.net.0.proj 4.6 -> 2.6 GB
- * of DRAM reads per launch; the Q projection reads least with 8). */
+ * of DRAM reads per launch; the Q projection reads least with 8).  Odd
+ * groups walk the N tiles in reverse, so each group starts on the weight
+ * tiles its predecessor read last. */
 constexpr int RASTER_SMALL_B = 8, RASTER_LARGE_B = 16;
 constexpr int64_t RASTER_LARGE_B_BYTES = 48ll << 20;
 /* mbarrier.try_wait suspend-time hints (ns): the producer and MMA threads wait
@@ -152,7 +154,9 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int ras
     const int gm = min(raster, num_m - first);
     const int r = t - g * per_group;
     mb = first + r % gm;
-    nb = r / gm;
+    /* odd groups walk N backwards: a group starts on the weight tiles the
+     * previous one ended on, which are still in L2 */
+    nb = (g & 1) ? num_n - 1 - r / gm : r / gm;
 }
 
 /*

@@ -182,7 +182,9 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int ras
     const int gm = min(raster, num_m - first);
     const int r = t - g * per_group;
     mb = first + r % gm;
-    nb = r / gm;
+    /* odd groups walk N backwards: a group starts on the weight tiles the
+     * previous one ended on, which are still in L2 */
+    nb = (g & 1) ? num_n - 1 - r / gm : r / gm;
 }
 
 /*
