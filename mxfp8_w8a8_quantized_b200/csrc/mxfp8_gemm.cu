@@ -60,6 +60,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <algorithm>
 #include <cstdint>
 #include <cstdlib>
 
@@ -75,12 +76,17 @@ constexpr int SF_WARP = 2 + EPI_WARPS; /* copies scales to TMEM (CTA-pair varian
 constexpr int GEMM_THREADS = (3 + EPI_WARPS) * 32;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0; /* 256 FP32 columns */
-/* M tiles walked together (for every N tile) so that their A rows stay in
- * L2: 8 when the weights fit in L2 alongside them, 16 when the weights are
- * re-read from DRAM once per group (measured: ffn.net.0.proj 4.6 -> 2.6 GB
- * of DRAM reads per launch; the Q projection reads least with 8).  Odd
- * groups walk the N tiles in reverse, so each group starts on the weight
- * tiles its predecessor read last. */
+/* Tile walk (tile_coords).  Preferred: groups of N tiles whose weight rows
+ * (at most RASTER_B_GROUP_BYTES) stay in L2 while the activation rows
+ * stream past them once per group -- used when such a group spans at least
+ * RASTER_MIN_N_GROUP N tiles.  Measured DRAM reads per launch at M = 75348
+ * (81 frames at 832x1104): N = K = 5120 705 -> 473 MB (the whole weight
+ * resident, A read once), ffn.net.0.proj 1.93 -> 1.58 GB.  Otherwise (long K:
+ * a weight tile is too large for a useful group) groups of M tiles walk every
+ * N tile: 8 when the weights fit in L2 alongside them, 16 when they are
+ * re-read from DRAM once per group. */
+constexpr int64_t RASTER_B_GROUP_BYTES = 48ll << 20;
+constexpr int RASTER_MIN_N_GROUP = 8;
 constexpr int RASTER_SMALL_B = 8, RASTER_LARGE_B = 16;
 constexpr int64_t RASTER_LARGE_B_BYTES = 48ll << 20;
 /* mbarrier.try_wait suspend-time hints (ns): the producer and MMA threads wait
@@ -142,21 +148,34 @@ struct GemmParams {
     int m_pad;            /* M rounded up to 128: rows that own scale bytes */
     int sf_kgroups;       /* N / 128: scale atoms per 128 output rows */
     int num_m, num_n;     /* output tiles */
-    int raster;           /* M tiles per raster group */
+    int raster;           /* > 0: M tiles per raster group; < 0: N tiles per group */
     unsigned long long timeout_ns;
 };
 
 __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int raster, int &mb, int &nb)
 {
-    const int per_group = raster * num_n;
-    const int g = t / per_group;
-    const int first = g * raster;
-    const int gm = min(raster, num_m - first);
-    const int r = t - g * per_group;
-    mb = first + r % gm;
-    /* odd groups walk N backwards: a group starts on the weight tiles the
-     * previous one ended on, which are still in L2 */
-    nb = (g & 1) ? num_n - 1 - r / gm : r / gm;
+    if (raster > 0) {
+        /* groups of `raster` M tiles, each group walked over every N tile */
+        const int per_group = raster * num_n;
+        const int g = t / per_group;
+        const int first = g * raster;
+        const int gm = min(raster, num_m - first);
+        const int r = t - g * per_group;
+        mb = first + r % gm;
+        /* odd groups walk N backwards: a group starts on the weight tiles the
+         * previous one ended on, which are still in L2 */
+        nb = (g & 1) ? num_n - 1 - r / gm : r / gm;
+    } else {
+        /* groups of -raster N tiles, each group walked over every M tile */
+        const int gsz = -raster;
+        const int per_group = gsz * num_m;
+        const int g = t / per_group;
+        const int first = g * gsz;
+        const int gn = min(gsz, num_n - first);
+        const int r = t - g * per_group;
+        nb = first + r % gn;
+        mb = (g & 1) ? num_m - 1 - r / gn : r / gn;
+    }
 }
 
 /*
@@ -934,7 +953,11 @@ int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void
     const int tile_m = pair ? Cfg<true>::TILE_M : Cfg<false>::TILE_M;
     p.num_m = (int)((M + tile_m - 1) / tile_m);
     p.num_n = (int)((N + 255) / 256);
-    p.raster = N * K > RASTER_LARGE_B_BYTES ? RASTER_LARGE_B : RASTER_SMALL_B;
+    const int64_t n_group = std::min<int64_t>(p.num_n, RASTER_B_GROUP_BYTES / ((int64_t)Cfg<true>::TILE_N * K));
+    if (n_group >= RASTER_MIN_N_GROUP)
+        p.raster = -(int)n_group;
+    else
+        p.raster = (int64_t)N * K > RASTER_LARGE_B_BYTES ? RASTER_LARGE_B : RASTER_SMALL_B;
     p.timeout_ns = timeout_ns;
     const int tiles = p.num_m * p.num_n;
     cudaError_t e;
