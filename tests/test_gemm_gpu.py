@@ -59,6 +59,26 @@ def test_linear_vs_oracle(mx, M, K, N):
     assert np.isfinite(y).all()
 
 
+# One shape per tile walk of the GEMM (groups of N tiles holding up to 48 MB
+# of weight rows when such a group spans at least 8 N tiles; else groups of
+# 8 M tiles, or 16 when the weights exceed 48 MB), each with several groups,
+# an odd group (walked in reverse) and a ragged last group.  Rows and columns
+# are sampled in every 128 x 128 quarter of every 256 x 256 tile, so a tile
+# the walk skipped or visited twice shows.
+@pytest.mark.parametrize("M,K,N", [
+    (300, 20480, 4864),    # N-tile groups of 9: 9 + 9 + 1 of 19 N tiles, two M tiles (ragged)
+    (2600, 256, 1024),     # M-tile groups of 8: 8 + 3 of 11 M tiles, four N tiles
+    (4400, 32768, 2048),   # M-tile groups of 16 (weights 67 MB): 16 + 2 of 18 M tiles
+])
+def test_tile_walk_covers_every_tile(mx, M, K, N):
+    x, w, b = make_layer(M, K, N, M + K)
+    y = gpu_linear(mx, x, w, b)
+    rows = sorted({min(r, M - 1) for t in range(0, M, 128) for r in (t, t + 77, t + 127)})
+    cols = sorted({min(c, N - 1) for t in range(0, N, 128) for c in (t, t + 50, t + 127)})
+    yref = oracle_linear(x, w, b, rows=np.array(rows), cols=np.array(cols))
+    assert_within_tol(y[np.ix_(rows, cols)], yref, f"tile walk {M}x{K}x{N}")
+
+
 def test_linear_without_bias(mx):
     x, w, _ = make_layer(200, 256, 264, 11, with_bias=False)
     y = gpu_linear(mx, x, w, None)
