@@ -57,6 +57,16 @@ __device__ __forceinline__ void load_seg16(Seg16<F32_IN> &s, const void *base, i
     }
 }
 
+/* max(|a|, |b|) of each BF16 half, two elements per instruction on the
+ * floating-point pipe (the integer pipe bounds this kernel at reduced SM
+ * clocks); the sign is the xor of the signs, a NaN gives the canonical NaN */
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 /* max |x| of the 16 elements, as the bit pattern of a binary32 (sign cleared) */
 template <bool F32_IN>
 __device__ __forceinline__ uint32_t amax_seg16(const Seg16<F32_IN> &s)
@@ -72,35 +82,43 @@ __device__ __forceinline__ uint32_t amax_seg16(const Seg16<F32_IN> &s)
         }
         return m;
     } else {
-        /* non-negative BF16 bit patterns order like the values (NaN above
-         * Inf above every finite value): packed unsigned 16-bit max */
-        const uint32_t k = 0x7FFF7FFFu;
-        uint32_t a = __vmaxu2(s.v[0].x & k, s.v[0].y & k);
-        uint32_t b = __vmaxu2(s.v[0].z & k, s.v[0].w & k);
-        uint32_t c = __vmaxu2(s.v[1].x & k, s.v[1].y & k);
-        uint32_t d = __vmaxu2(s.v[1].z & k, s.v[1].w & k);
-        uint32_t m = __vmaxu2(__vmaxu2(a, b), __vmaxu2(c, d));
+        /* per half, the largest magnitude (a NaN anywhere gives the canonical
+         * NaN, whose exponent field marks the block as non-finite) */
+        const uint32_t a = absmax_bf16x2(s.v[0].x, s.v[0].y);
+        const uint32_t b = absmax_bf16x2(s.v[0].z, s.v[0].w);
+        const uint32_t c = absmax_bf16x2(s.v[1].x, s.v[1].y);
+        const uint32_t d = absmax_bf16x2(s.v[1].z, s.v[1].w);
+        const uint32_t m = absmax_bf16x2(absmax_bf16x2(a, b), absmax_bf16x2(c, d)) & 0x7FFF7FFFu;
+        /* non-negative BF16 bit patterns order like the values */
         return max(m << 16, m & 0xFFFF0000u);
     }
 }
 
-/* 16 elements times 2^-e (exact) -> 16 E4M3 codes */
+/* 16 elements times 2^-e (exact) -> 16 E4M3 codes; `sb` is the block's
+ * finite scale byte (e = sb - 127, sb <= 246).  The BF16 path multiplies
+ * pairs with one packed binary32 instruction (each lane rounded like the
+ * scalar multiply, which is exact here). */
 template <bool F32_IN>
-__device__ __forceinline__ uint4 codes_seg16(const Seg16<F32_IN> &s, float m)
+__device__ __forceinline__ uint4 codes_seg16(const Seg16<F32_IN> &s, uint32_t sb)
 {
     uint32_t out[4];
     if constexpr (F32_IN) {
+        const float m = inv_scale(sb);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
             out[i] = pack4_e4m3(__uint_as_float(s.v[i].x) * m, __uint_as_float(s.v[i].y) * m,
                                 __uint_as_float(s.v[i].z) * m, __uint_as_float(s.v[i].w) * m);
     } else {
+        const float m = inv_scale(sb);
+        const f32x2 mm = f2_pack(m, m);
         const uint32_t w[8] = {s.v[0].x, s.v[0].y, s.v[0].z, s.v[0].w, s.v[1].x, s.v[1].y, s.v[1].z, s.v[1].w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            out[i] = pack4_e4m3(__uint_as_float(w[2 * i] << 16) * m, __uint_as_float(w[2 * i] & 0xFFFF0000u) * m,
-                                __uint_as_float(w[2 * i + 1] << 16) * m,
-                                __uint_as_float(w[2 * i + 1] & 0xFFFF0000u) * m);
+        for (int i = 0; i < 4; ++i) {
+            float c0, c1, c2, c3;
+            f2_unpack(f2_mul(bf16x2_to_f32x2(w[2 * i]), mm), c0, c1);
+            f2_unpack(f2_mul(bf16x2_to_f32x2(w[2 * i + 1]), mm), c2, c3);
+            out[i] = pack4_e4m3(c0, c1, c2, c3);
+        }
     }
     return make_uint4(out[0], out[1], out[2], out[3]);
 }
@@ -166,7 +184,7 @@ __global__ void __launch_bounds__(QTHREADS, 1) mx_quantize_kernel(const void *__
             const uint32_t sb = valid[i] ? scale_byte_from_amax(amax) : 0u;
             if (valid[i]) {
                 const uint4 out = (sb == 0xFFu) ? make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu)
-                                                : codes_seg16<F32_IN>(seg[i], inv_scale(sb));
+                                                : codes_seg16<F32_IN>(seg[i], sb);
                 *reinterpret_cast<uint4 *>(Q + (int64_t)row[i] * K + k0[i]) = out;
             }
             if constexpr (SF_TC) {
