@@ -14,15 +14,17 @@
  * x * 2^-e (exact: a power-of-two multiply of a BF16/FP32 value).
  *
  * HBM-bound: 2 (BF16) or 4 (FP32) bytes read + 1 code byte + 1/32 scale byte
- * written per element.  Each warp handles row segments of 512 elements: every
- * lane loads 16 consecutive elements with two 128-bit loads (fully coalesced),
- * two lanes form one 32-block and combine their amax with one shuffle, each
- * lane writes its 16 codes with one 16-byte store (coalesced 512 B per warp),
- * and scales are gathered into 32-bit words written straight into the
- * tensor-core scale layout (see include/mxfp8.h).  Two segments are loaded
- * before either is processed, keeping four 16-byte loads in flight per
- * thread.  The row/segment walk has no division in the loop: the kernel is
- * close to instruction-bound, so every per-element instruction counts.
+ * written per element.  Each warp walks whole rows in segments of 512
+ * elements: every lane loads 16 consecutive elements with two 128-bit loads
+ * (fully coalesced), two lanes form one 32-block and combine their amax with
+ * one shuffle, each lane writes its 16 codes with one 16-byte store
+ * (coalesced 512 B per warp), and scales are gathered into 32-bit words
+ * written straight into the tensor-core scale layout (see include/mxfp8.h).
+ * Two segments are loaded before either is processed, keeping four 16-byte
+ * loads in flight per thread.  At the SM clocks of a power-capped GPU the
+ * kernel is close to bound by its integer instructions, so every address in a
+ * row is the row's base plus a multiple of the segment, and the block amax
+ * and the scaling run on the floating-point pipe, two elements at a time.
  */
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
@@ -42,19 +44,14 @@ struct Seg16 {
     uint4 v[F32_IN ? 4 : 2];
 };
 
+/* the 16 elements of a row starting at element k0 (streaming loads) */
 template <bool F32_IN>
-__device__ __forceinline__ void load_seg16(Seg16<F32_IN> &s, const void *base, int64_t elem_off)
+__device__ __forceinline__ void load_seg16(Seg16<F32_IN> &s, const uint8_t *row, int k0)
 {
-    if constexpr (F32_IN) {
-        const uint4 *p = reinterpret_cast<const uint4 *>(reinterpret_cast<const float *>(base) + elem_off);
+    const uint4 *p = reinterpret_cast<const uint4 *>(row + (int64_t)k0 * (F32_IN ? 4 : 2));
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            s.v[i] = __ldcs(p + i);
-    } else {
-        const uint4 *p = reinterpret_cast<const uint4 *>(reinterpret_cast<const uint16_t *>(base) + elem_off);
-        s.v[0] = __ldcs(p);
-        s.v[1] = __ldcs(p + 1);
-    }
+    for (int i = 0; i < (F32_IN ? 4 : 2); ++i)
+        s.v[i] = __ldcs(p + i);
 }
 
 /* max(|a|, |b|) of each BF16 half, two elements per instruction on the
@@ -125,9 +122,11 @@ __device__ __forceinline__ uint4 codes_seg16(const Seg16<F32_IN> &s, uint32_t sb
 
 /*
  * X [M, K] (row stride ldx elements) -> Q [M, K] codes, S scales.
- * Work unit = (row r, segment j of 512 elements); lane l covers elements
- * 16l .. 16l+15 of the segment, so lanes 2b and 2b+1 hold block b.  Rows r in
- * [M, Mrows) only write zero scale padding (tensor-core layout).
+ * Each warp walks whole rows (rows warp, warp + nwarps, ...), two 512-element
+ * segments at a time; lane l covers elements 16l .. 16l+15 of a segment, so
+ * lanes 2b and 2b+1 hold block b.  Every address of a row is its base plus a
+ * multiple of the segment.  Rows r in [M, Mrows) only write zero scale
+ * padding (tensor-core layout).
  */
 template <bool F32_IN, bool SF_TC>
 __global__ void __launch_bounds__(QTHREADS, 1) mx_quantize_kernel(const void *__restrict__ X, int64_t M,
@@ -137,73 +136,53 @@ __global__ void __launch_bounds__(QTHREADS, 1) mx_quantize_kernel(const void *__
                                                                               int64_t nseg, int64_t kgroups)
 {
     const int lane = threadIdx.x & 31;
-    const int64_t warp0 = ((int64_t)blockIdx.x * QTHREADS + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * QTHREADS) >> 5;
-    const int64_t units = Mrows * nseg;
+    const int warp0 = (int)((blockIdx.x * QTHREADS + threadIdx.x) >> 5);
+    const int nwarps = (int)((gridDim.x * QTHREADS) >> 5);
     const int nblocks = (int)(K >> 5);
-    /* Walk the (row, segment) space without dividing in the loop: one
-     * division up front, then carry-propagating increments. */
-    const int64_t stride = nwarps * QUNROLL;
-    const int nseg32 = (int)nseg;
-    const int stride_r = (int)(stride / nseg), stride_j = (int)(stride - (int64_t)stride_r * nseg);
-    int64_t u0 = warp0 * QUNROLL;
-    int r0 = (int)(u0 / nseg), j0 = (int)(u0 - (int64_t)r0 * nseg);
-    const int M32 = (int)M, K32 = (int)K;
+    const int M32 = (int)M, K32 = (int)K, nseg32 = (int)nseg, Mrows32 = (int)Mrows;
+    constexpr int EB = F32_IN ? 4 : 2;
 
-    for (; u0 < units; u0 += stride) {
-        Seg16<F32_IN> seg[QUNROLL];
-        int row[QUNROLL], k0[QUNROLL];
-        bool valid[QUNROLL];
-        {
-            int r = r0, j = j0;
+    for (int r = warp0; r < Mrows32; r += nwarps) {
+        const bool row_ok = r < M32;
+        const uint8_t *xrow = reinterpret_cast<const uint8_t *>(X) + (int64_t)r * ldx * EB;
+        uint8_t *qrow = Q + (int64_t)r * K;
+        uint8_t *srow = SF_TC ? S + ((((int64_t)(r >> 7)) * kgroups) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2)
+                              : S + (int64_t)r * nblocks;
+        for (int j = 0; j < nseg32; j += QUNROLL) {
+            Seg16<F32_IN> seg[QUNROLL];
+            int k0[QUNROLL];
+            bool valid[QUNROLL];
 #pragma unroll
             for (int i = 0; i < QUNROLL; ++i) {
-                row[i] = r;
-                k0[i] = j * 512 + lane * 16;
-                valid[i] = (u0 + i < units) && (r < M32) && (k0[i] < K32);
+                k0[i] = (j + i) * 512 + lane * 16;
+                valid[i] = row_ok && (j + i < nseg32) && (k0[i] < K32);
                 if (valid[i])
-                    load_seg16<F32_IN>(seg[i], X, (int64_t)r * ldx + k0[i]);
-                if (++j == nseg32) {
-                    j = 0;
-                    ++r;
-                }
+                    load_seg16<F32_IN>(seg[i], xrow, k0[i]);
             }
-        }
-        r0 += stride_r;
-        j0 += stride_j;
-        if (j0 >= nseg32) {
-            j0 -= nseg32;
-            ++r0;
-        }
 #pragma unroll
-        for (int i = 0; i < QUNROLL; ++i) {
-            if (u0 + i >= units) /* warp-uniform */
-                break;
-            uint32_t amax = valid[i] ? amax_seg16<F32_IN>(seg[i]) : 0u;
-            amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-            const uint32_t sb = valid[i] ? scale_byte_from_amax(amax) : 0u;
-            if (valid[i]) {
-                const uint4 out = (sb == 0xFFu) ? make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu)
-                                                : codes_seg16<F32_IN>(seg[i], sb);
-                *reinterpret_cast<uint4 *>(Q + (int64_t)row[i] * K + k0[i]) = out;
-            }
-            if constexpr (SF_TC) {
-                /* word g (lanes 8g .. 8g+7) = blocks 16j + 4g .. 16j + 4g + 3 */
-                const uint32_t w = sb | (__shfl_down_sync(0xFFFFFFFFu, sb, 2) << 8) |
-                                   (__shfl_down_sync(0xFFFFFFFFu, sb, 4) << 16) |
-                                   (__shfl_down_sync(0xFFFFFFFFu, sb, 6) << 24);
-                if ((lane & 7) == 0) {
-                    const int r = row[i];
-                    const int kb = ((k0[i] - lane * 16) >> 5) + (lane >> 1); /* first block of this word */
-                    if (kb < nblocks) {
-                        const int64_t off = ((((int64_t)(r >> 7)) * kgroups + (kb >> 2)) << 9) + ((r & 31) << 4) +
-                                            (((r >> 5) & 3) << 2);
-                        *reinterpret_cast<uint32_t *>(S + off) = w;
-                    }
+            for (int i = 0; i < QUNROLL; ++i) {
+                if (j + i >= nseg32) /* warp-uniform */
+                    break;
+                uint32_t amax = valid[i] ? amax_seg16<F32_IN>(seg[i]) : 0u;
+                amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+                const uint32_t sb = valid[i] ? scale_byte_from_amax(amax) : 0u;
+                if (valid[i]) {
+                    const uint4 out = (sb == 0xFFu) ? make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu)
+                                                    : codes_seg16<F32_IN>(seg[i], sb);
+                    *reinterpret_cast<uint4 *>(qrow + k0[i]) = out;
                 }
-            } else {
-                if (valid[i] && (lane & 1) == 0)
-                    S[(int64_t)row[i] * nblocks + (k0[i] >> 5)] = (uint8_t)sb;
+                if constexpr (SF_TC) {
+                    /* word g (lanes 8g .. 8g+7) = blocks 16(j+i) + 4g .. 16(j+i) + 4g + 3 */
+                    const uint32_t w = sb | (__shfl_down_sync(0xFFFFFFFFu, sb, 2) << 8) |
+                                       (__shfl_down_sync(0xFFFFFFFFu, sb, 4) << 16) |
+                                       (__shfl_down_sync(0xFFFFFFFFu, sb, 6) << 24);
+                    const int kb = (j + i) * 16 + (lane >> 1); /* first block of this word */
+                    if ((lane & 7) == 0 && kb < nblocks)
+                        *reinterpret_cast<uint32_t *>(srow + ((int64_t)(kb >> 2) << 9)) = w;
+                } else {
+                    if (valid[i] && (lane & 1) == 0)
+                        srow[k0[i] >> 5] = (uint8_t)sb;
+                }
             }
         }
     }
@@ -247,8 +226,8 @@ cudaError_t launch_quantize(const void *X, bool f32_in, int64_t M, int64_t K, in
     const int64_t units = Mrows * nseg;
     if (units == 0)
         return cudaSuccess;
-    const int64_t per_block = (QTHREADS / 32) * QUNROLL;
-    int64_t blocks = (units + per_block - 1) / per_block;
+    const int64_t per_block = QTHREADS / 32; /* rows per block */
+    int64_t blocks = (Mrows + per_block - 1) / per_block;
     const int64_t cap = (int64_t)num_sms_cached() * 8 * 4; /* 8 resident blocks x 4 waves */
     if (blocks > cap)
         blocks = cap;
