@@ -15,10 +15,12 @@
  *
  * HBM-bound: 2 (BF16) or 4 (FP32) bytes read, 0.5 + 1/16 byte written per
  * element.  One lane owns one block (16 elements, two 16-byte loads), so the
- * block amax needs no shuffle; a warp covers 512 elements of a row; four
- * lanes' scale bytes form one 32-bit word of an atom.  Two segments are in
- * flight per warp and the row / segment walk has no division in the loop.
- * FP32 weights are rounded to BF16 (nearest even) on load.
+ * block amax needs no shuffle; each warp walks whole rows in segments of 512
+ * elements (every address in a row is the row's base plus a multiple of the
+ * segment), two segments in flight; four lanes' scale bytes form one 32-bit
+ * word of an atom.  The block amax and the scaling run two elements per
+ * instruction on the floating-point pipe.  FP32 weights are rounded to BF16
+ * (nearest even) on load.
  */
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -26,17 +28,19 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "mx_element.cuh"
+
 namespace mx {
 
 constexpr int NQ_THREADS = 256;
 constexpr int NQ_UNROLL = 2;
 
-/* 16 elements of a row as 8 words of BF16 pairs. */
+/* the 16 elements starting at element k0 of `row`, as 8 words of BF16 pairs */
 template <bool F32_IN>
-__device__ __forceinline__ void nq_load16(uint32_t (&w)[8], const void *base, int64_t elem_off)
+__device__ __forceinline__ void nq_load16(uint32_t (&w)[8], const uint8_t *row, int64_t k0)
 {
     if constexpr (F32_IN) {
-        const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const float *>(base) + elem_off);
+        const uint4 *p = reinterpret_cast<const uint4 *>(row + k0 * 4);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const uint4 v = __ldcs(p + i);
@@ -46,10 +50,19 @@ __device__ __forceinline__ void nq_load16(uint32_t (&w)[8], const void *base, in
             w[2 * i + 1] = *reinterpret_cast<uint32_t *>(&b);
         }
     } else {
-        const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(base) + elem_off);
+        const uint4 *p = reinterpret_cast<const uint4 *>(row + k0 * 2);
         const uint4 a = __ldcs(p), b = __ldcs(p + 1);
         w[0] = a.x, w[1] = a.y, w[2] = a.z, w[3] = a.w, w[4] = b.x, w[5] = b.y, w[6] = b.z, w[7] = b.w;
     }
+}
+
+/* max(|a|, |b|) of each BF16 half (sign = xor of the signs; a NaN gives the
+ * canonical NaN) */
+__device__ __forceinline__ uint32_t nq_absmax_bf16x2(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
 }
 
 /* 8 values -> 4 bytes of E2M1 pairs (even element in the low nibble). */
@@ -70,9 +83,9 @@ __device__ __forceinline__ uint32_t nq_e2m1x8(float x0, float x1, float x2, floa
 
 /*
  * X [M, K] (row stride ldx) -> Q [M, K/2] packed codes, S scales (tensor-core
- * layout, kg = ceil(K / 64) atoms per 128 rows).  Work unit = (row r,
- * segment j of 512 elements); lane l owns block 32 j + l.  Rows in [M, Mrows)
- * only write zero scale padding.
+ * layout, kg = ceil(K / 64) atoms per 128 rows).  Each warp walks whole rows
+ * (rows warp, warp + nwarps, ...); in segment j lane l owns block 32 j + l.
+ * Rows in [M, Mrows) only write zero scale padding.
  */
 template <bool F32_IN>
 __global__ void __launch_bounds__(NQ_THREADS) nvfp4_quantize_kernel(const void *__restrict__ X, int64_t M, int64_t K,
@@ -82,82 +95,64 @@ __global__ void __launch_bounds__(NQ_THREADS) nvfp4_quantize_kernel(const void *
                                                                     int64_t nseg, int64_t kg)
 {
     const int lane = threadIdx.x & 31;
-    const int64_t warp0 = ((int64_t)blockIdx.x * NQ_THREADS + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * NQ_THREADS) >> 5;
-    const int64_t units = Mrows * nseg;
+    const int warp0 = (int)((blockIdx.x * NQ_THREADS + threadIdx.x) >> 5);
+    const int nwarps = (int)((gridDim.x * NQ_THREADS) >> 5);
     const int nblocks = (int)(K >> 4);
     const float g = __ldg(gptr);
     const float gs = __fdiv_rn(g, 6.0f);
-    const int64_t stride = nwarps * NQ_UNROLL;
-    const int nseg32 = (int)nseg;
-    const int stride_r = (int)(stride / nseg), stride_j = (int)(stride - (int64_t)stride_r * nseg);
-    int64_t u0 = warp0 * NQ_UNROLL;
-    int r0 = (int)(u0 / nseg), j0 = (int)(u0 - (int64_t)r0 * nseg);
-    const int M32 = (int)M, K32 = (int)K;
+    const int M32 = (int)M, K32 = (int)K, nseg32 = (int)nseg, Mrows32 = (int)Mrows;
+    constexpr int EB = F32_IN ? 4 : 2;
 
-    for (; u0 < units; u0 += stride) {
-        uint32_t w[NQ_UNROLL][8];
-        int row[NQ_UNROLL], k0[NQ_UNROLL];
-        bool valid[NQ_UNROLL];
-        {
-            int r = r0, j = j0;
+    for (int r = warp0; r < Mrows32; r += nwarps) {
+        const bool row_ok = r < M32;
+        const uint8_t *xrow = reinterpret_cast<const uint8_t *>(X) + (int64_t)r * ldx * EB;
+        uint8_t *qrow = Q + (int64_t)r * (K >> 1);
+        uint8_t *srow = S + ((((int64_t)(r >> 7)) * kg) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2);
+        for (int j = 0; j < nseg32; j += NQ_UNROLL) {
+            uint32_t w[NQ_UNROLL][8];
+            int k0[NQ_UNROLL];
+            bool valid[NQ_UNROLL];
 #pragma unroll
             for (int i = 0; i < NQ_UNROLL; ++i) {
-                row[i] = r;
-                k0[i] = j * 512 + lane * 16;
-                valid[i] = (u0 + i < units) && (r < M32) && (k0[i] < K32);
+                k0[i] = (j + i) * 512 + lane * 16;
+                valid[i] = row_ok && (j + i < nseg32) && (k0[i] < K32);
                 if (valid[i])
-                    nq_load16<F32_IN>(w[i], X, (int64_t)r * ldx + k0[i]);
-                if (++j == nseg32) {
-                    j = 0;
-                    ++r;
-                }
+                    nq_load16<F32_IN>(w[i], xrow, k0[i]);
             }
-        }
-        r0 += stride_r;
-        j0 += stride_j;
-        if (j0 >= nseg32) {
-            j0 -= nseg32;
-            ++r0;
-        }
 #pragma unroll
-        for (int i = 0; i < NQ_UNROLL; ++i) {
-            if (u0 + i >= units) /* warp-uniform */
-                break;
-            uint32_t sb = 0u;
-            if (valid[i]) {
-                /* non-negative BF16 bit patterns order like their values */
-                uint32_t m2 = 0u;
+            for (int i = 0; i < NQ_UNROLL; ++i) {
+                if (j + i >= nseg32) /* warp-uniform */
+                    break;
+                uint32_t sb = 0u;
+                if (valid[i]) {
+                    const uint32_t a = nq_absmax_bf16x2(w[i][0], w[i][1]);
+                    const uint32_t b = nq_absmax_bf16x2(w[i][2], w[i][3]);
+                    const uint32_t c = nq_absmax_bf16x2(w[i][4], w[i][5]);
+                    const uint32_t d = nq_absmax_bf16x2(w[i][6], w[i][7]);
+                    const uint32_t m2 = nq_absmax_bf16x2(nq_absmax_bf16x2(a, b), nq_absmax_bf16x2(c, d)) & 0x7FFF7FFFu;
+                    /* non-negative BF16 bit patterns order like their values */
+                    const float amax = __uint_as_float(max(m2 << 16, m2 & 0xFFFF0000u));
+                    sb = (uint32_t)__nv_cvt_float_to_fp8(amax * gs, __NV_SATFINITE, __NV_E4M3) & 0x7Fu;
+                    const __half_raw hr = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)sb, __NV_E4M3);
+                    const float ds = __half2float(__half(hr));
+                    const float mul = ds > 0.0f ? __fdiv_rn(g, ds) : 0.0f;
+                    /* packed binary32 multiplies: each lane rounded like the scalar one */
+                    const f32x2 mm = f2_pack(mul, mul);
+                    float f[16];
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    m2 = __vmaxu2(m2, w[i][k] & 0x7FFF7FFFu);
-                const float amax = __uint_as_float(max(m2 << 16, m2 & 0xFFFF0000u));
-                sb = (uint32_t)__nv_cvt_float_to_fp8(amax * gs, __NV_SATFINITE, __NV_E4M3) & 0x7Fu;
-                const __half_raw hr = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)sb, __NV_E4M3);
-                const float ds = __half2float(__half(hr));
-                const float mul = ds > 0.0f ? __fdiv_rn(g, ds) : 0.0f;
-                float f[16];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    f[2 * k] = __uint_as_float(w[i][k] << 16) * mul;
-                    f[2 * k + 1] = __uint_as_float(w[i][k] & 0xFFFF0000u) * mul;
+                    for (int k = 0; k < 8; ++k)
+                        f2_unpack(f2_mul(bf16x2_to_f32x2(w[i][k]), mm), f[2 * k], f[2 * k + 1]);
+                    const uint32_t lo = nq_e2m1x8(f[0], f[1], f[2], f[3], f[4], f[5], f[6], f[7]);
+                    const uint32_t hi = nq_e2m1x8(f[8], f[9], f[10], f[11], f[12], f[13], f[14], f[15]);
+                    *reinterpret_cast<uint2 *>(qrow + (k0[i] >> 1)) = make_uint2(lo, hi);
                 }
-                const uint32_t lo = nq_e2m1x8(f[0], f[1], f[2], f[3], f[4], f[5], f[6], f[7]);
-                const uint32_t hi = nq_e2m1x8(f[8], f[9], f[10], f[11], f[12], f[13], f[14], f[15]);
-                *reinterpret_cast<uint2 *>(Q + (int64_t)row[i] * (K >> 1) + (k0[i] >> 1)) = make_uint2(lo, hi);
-            }
-            /* word g (lanes 4g .. 4g+3) = blocks 32 j + 4g .. 32 j + 4g + 3 */
-            const uint32_t word = sb | (__shfl_down_sync(0xFFFFFFFFu, sb, 1) << 8) |
-                                  (__shfl_down_sync(0xFFFFFFFFu, sb, 2) << 16) |
-                                  (__shfl_down_sync(0xFFFFFFFFu, sb, 3) << 24);
-            if ((lane & 3) == 0) {
-                const int r = row[i];
-                const int b = (k0[i] >> 4); /* this lane's block = first block of the word */
-                if (b < nblocks) {
-                    const int64_t off = ((((int64_t)(r >> 7)) * kg + (b >> 2)) << 9) + ((r & 31) << 4) +
-                                        (((r >> 5) & 3) << 2);
-                    *reinterpret_cast<uint32_t *>(S + off) = word;
-                }
+                /* word q (lanes 4q .. 4q+3) = blocks 32 (j+i) + 4q .. 32 (j+i) + 4q + 3 */
+                const uint32_t word = sb | (__shfl_down_sync(0xFFFFFFFFu, sb, 1) << 8) |
+                                      (__shfl_down_sync(0xFFFFFFFFu, sb, 2) << 16) |
+                                      (__shfl_down_sync(0xFFFFFFFFu, sb, 3) << 24);
+                const int bk = k0[i] >> 4; /* this lane's block = first block of the word */
+                if ((lane & 3) == 0 && bk < nblocks)
+                    *reinterpret_cast<uint32_t *>(srow + ((int64_t)(bk >> 2) << 9)) = word;
             }
         }
     }
@@ -172,7 +167,7 @@ __global__ void __launch_bounds__(256) nvfp4_amax_kernel(const void *__restrict_
     uint32_t m2 = 0u;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += (int64_t)gridDim.x * blockDim.x) {
         uint32_t w[8];
-        nq_load16<F32_IN>(w, X, i * 16);
+        nq_load16<F32_IN>(w, reinterpret_cast<const uint8_t *>(X), i * 16);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
             m2 = __vmaxu2(m2, w[k] & 0x7FFF7FFFu);
@@ -222,8 +217,8 @@ cudaError_t launch_nvfp4_quantize(const void *X, bool f32_in, int64_t M, int64_t
     const int64_t units = Mrows * nseg;
     if (units == 0)
         return cudaSuccess;
-    const int64_t per_block = (NQ_THREADS / 32) * NQ_UNROLL;
-    int64_t blocks = (units + per_block - 1) / per_block;
+    const int64_t per_block = NQ_THREADS / 32; /* rows per block */
+    int64_t blocks = (Mrows + per_block - 1) / per_block;
     const int64_t cap = (int64_t)nq_num_sms() * 8 * 4; /* 8 resident blocks x 4 waves */
     if (blocks > cap)
         blocks = cap;
