@@ -50,7 +50,10 @@ def test_global_scale_on_device(mx):
         assert float(rg) == g and dg.item() == g
 
 
-@pytest.mark.parametrize("M,K", [(256, 512), (1, 16), (300, 5120), (129, 13824), (1000, 1040), (64, 48)])
+# (40000, 48): more rows than the quantizer's resident warps (32 x 148
+# blocks x 8), so warps walk a second row; three blocks per row.
+@pytest.mark.parametrize("M,K", [(256, 512), (1, 16), (300, 5120), (129, 13824), (1000, 1040), (64, 48),
+                                 (40000, 48)])
 def test_activation_quantizer_bit_exact(mx, M, K):
     x = synth.activations_device(M, K, M + K, 0, "cuda")
     g, g_ref = _g(mx, x)

@@ -41,8 +41,10 @@ def check_act(mx, x_cpu, what):
     assert (s2[~used] == 0).all(), f"{what}: padding not zero"
 
 
+# (40000, 96): more rows than the quantizer's resident warps (32 x 148
+# blocks x 8), so warps walk a second row; one partial segment per row.
 @pytest.mark.parametrize("M,K", [(256, 512), (1, 32), (7, 96), (129, 256), (300, 160), (128, 5120),
-                                 (37, 13824), (1000, 640)])
+                                 (37, 13824), (1000, 640), (40000, 96)])
 def test_activation_quant_workload_distribution(mx, M, K):
     x = synth.activations(M, K, seed=M + K)
     check_act(mx, x, f"M={M} K={K}")
