@@ -39,6 +39,7 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_BF16_SUSTAINED = 1400.0
 FP8_OVER_BF16 = 2.0  # nominal dense ratio: 4.5 PF/s FP8 vs 2.25 PF/s BF16
+FP4_OVER_BF16 = 4.0  # nominal dense ratio: 9 PF/s FP4 vs 2.25 PF/s BF16
 L2_FLUSH_BYTES = 256 << 20
 WORKLOADS = ["c4_step_832x1104", "c1_q_proj_480p", "c0_small", "ffn0_832x1104", "ffn2_832x1104",
              "c2_ffn_pair_832x1104", "c3_block_832x1104"]
@@ -347,11 +348,11 @@ class NVFP4LinearWorkload(LinearWorkload):
     scale is a calibrated constant of the layer, not computed per step)."""
 
     scheme = "nvfp4"
-    gemm_kernel = "nvfp4_gemm_kernel"
+    gemm_kernel = "mxfp8_gemm_kernel"     # its NVFP4 mode: tcgen05.mma kind::mxf4nvf4
     quant_kernel = "nvfp4_quantize_kernel"
-    profile_kernel = "nvfp4_gemm"
-    tc_over_bf16 = 1.0    # the codes are expanded to FP16: the FP16 tensor-core rate (= BF16)
-    dtype = "e2m1 + ue4m3/16 (NVFP4 operands expanded exactly to fp16 for the tensor core), fp32 accumulate, " \
+    profile_kernel = "mxfp8_gemm"
+    tc_over_bf16 = FP4_OVER_BF16
+    dtype = "e2m1 + ue4m3/16 (NVFP4 operands on the 4-bit block-scaled tensor-core kind), fp32 accumulate, " \
             "bf16 out"
 
     def config(self):
@@ -668,9 +669,8 @@ def run_ours(args, ranks, dev):
         "roofline": {"bound": "tensor", "kernel": wl.gemm_kernel,
                      "achieved": round(gemm_tflops, 1), "peak": round(tc_peak, 1), "unit": "TFLOP/s",
                      "frac": round(gemm_tflops / tc_peak, 4),
-                     "peak_source": (f"{peak_src} bf16 {kind} x {FP8_OVER_BF16} (nominal FP8/BF16 ratio)"
-                                     if wl.tc_over_bf16 != 1.0 else
-                                     f"{peak_src} bf16 {kind} (the FP16 kind runs at the BF16 rate)"),
+                     "peak_source": f"{peak_src} bf16 {kind} x {wl.tc_over_bf16} (nominal "
+                                    f"{'FP4' if wl.tc_over_bf16 == FP4_OVER_BF16 else 'FP8'}/BF16 ratio)",
                      "traffic": load_traffic(wl.profile_key, wl.profile_kernel),
                      "algorithmic_bytes_per_step": round(wl.gemm_bytes()),
                      "launches_per_step": g_n // kernel_steps, "avg_launch_ms": round(g_ms / g_n, 4)},

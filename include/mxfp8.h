@@ -226,8 +226,8 @@ mxfp8_status mxfp8_device_status(mxfp8_stream_t stream);
 
 /* Which kernel family's bounded wait mxfp8_selftest_wait_timeout exercises. */
 typedef enum {
-    MXFP8_SELFTEST_GEMM = 0,           /* the MXFP8 / per-channel FP8 GEMM */
-    MXFP8_SELFTEST_NVFP4_GEMM = 1,     /* the NVFP4 GEMM */
+    MXFP8_SELFTEST_GEMM = 0,           /* the block-scaled / per-channel FP8 GEMM */
+    MXFP8_SELFTEST_NVFP4_GEMM = 1,     /* the NVFP4 GEMM: the same kernel family and wait as 0 */
     MXFP8_SELFTEST_ROWWISE_QUANT = 2   /* the per-channel FP8 activation quantizer */
 } mxfp8_selftest;
 

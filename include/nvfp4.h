@@ -14,11 +14,11 @@
  *                                       s = 0 gives q = +-0
  *   dequantized value q * dec(s) / g; the layer computes
  *     Y[m, n] = BF16_RNE(alpha * sum_k (qx dec(sx)) (qw dec(sw)) + F32(bias[n]))
- *   with alpha = 1 / (g_x * g_w) and FP32 accumulation.  Each product
- *   q * dec(s) is exact in FP16 (at most 6 significant bits), so the GEMM
- *   expands the codes to FP16 in the SM and runs on the FP16 tensor-core
- *   kind; the sum is that of a block-scaled 4-bit MMA up to the order of
- *   the FP32 additions.
+ *   with alpha = 1 / (g_x * g_w) and FP32 accumulation.  The GEMM runs the
+ *   block-scaled 4-bit tensor-core kind (tcgen05.mma kind::mxf4nvf4,
+ *   16-element UE4M3 scales): the packed codes are its operands as stored
+ *   and the scale atoms below are its scale layout; the epilogue applies
+ *   alpha and the bias.
  *
  * Global scales live in device memory (one binary32 per tensor), so the
  * whole path runs on the GPU with no host round trip: nvfp4_amax_* measures

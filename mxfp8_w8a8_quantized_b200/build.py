@@ -17,14 +17,12 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmxfp8.so")
 
 PUBLIC_HEADERS = ["mxfp8.h", "fp8_rowwise.h", "nvfp4.h"]
-SOURCES = ["mxfp8_quant.cu", "mxfp8_gemm.cu", "mxfp8_capi.cu", "mxfp8_noalloc.cu", "fp8_rowwise.cu", "nvfp4.cu",
-           "nvfp4_gemm.cu"]
+SOURCES = ["mxfp8_quant.cu", "mxfp8_gemm.cu", "mxfp8_capi.cu", "mxfp8_noalloc.cu", "fp8_rowwise.cu", "nvfp4.cu"]
 HEADERS = ["ptx.cuh", "mx_element.cuh", "tmap_host.cuh"]
 # The files each profiled kernel is compiled from: a profile summary names
 # the hash of its kernel's files, so that it goes stale only when they change.
 KERNEL_FILES = {
     "mxfp8_gemm": ["mxfp8_gemm.cu", "ptx.cuh", "mx_element.cuh", "tmap_host.cuh"],
-    "nvfp4_gemm": ["nvfp4_gemm.cu", "ptx.cuh", "tmap_host.cuh"],
 }
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -15,7 +15,7 @@ cudaError_t launch_quantize(const void *X, bool f32_in, int64_t M, int64_t K, in
 cudaError_t launch_gelu(const void *X, void *Y, int64_t n, cudaStream_t stream);
 int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void *Wq, const void *Ws, int64_t N,
                 const void *bias, void *Y, int epi, void *S, cudaStream_t stream, unsigned long long timeout_ns,
-                cudaError_t *err);
+                cudaError_t *err, const float *gx = nullptr, const float *gw = nullptr);
 cudaError_t launch_nvfp4_quantize(const void *X, bool f32_in, int64_t M, int64_t K, int64_t ldx, const float *g,
                                   uint8_t *Q, uint8_t *S, cudaStream_t stream);
 cudaError_t launch_nvfp4_amax(const void *X, bool f32_in, int64_t n, unsigned int *out, cudaStream_t stream);
@@ -24,12 +24,7 @@ cudaError_t read_and_clear_status(unsigned int *out);
 cudaError_t launch_fp8_rowwise_quantize(const void *X, bool f32_in, int64_t M, int64_t K, int64_t ldx, uint8_t *Q,
                                         float *S, cudaStream_t stream, unsigned long long timeout_ns);
 cudaError_t read_and_clear_rw_status(unsigned int *out);
-int launch_nvfp4_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void *Wq, const void *Ws,
-                      int64_t N, const float *gx, const float *gw, const void *bias, void *Y,
-                      cudaStream_t stream, unsigned long long timeout_ns, cudaError_t *err);
-cudaError_t read_and_clear_nv_status(unsigned int *out);
 cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t stream);
-cudaError_t launch_nv_wait_selftest(unsigned long long limit_ns, cudaStream_t stream);
 cudaError_t launch_rw_wait_selftest(unsigned long long limit_ns, cudaStream_t stream);
 } // namespace mx
 
@@ -412,8 +407,9 @@ mxfp8_status nvfp4_gemm(const void *Xq, const void *Xscale, int64_t M, int64_t K
     if (st != MXFP8_OK || M == 0)
         return st;
     cudaError_t e;
-    int r = mx::launch_nvfp4_gemm(Xq, Xscale, M, K, Wq, Wscale, N, x_global_scale, w_global_scale, bias, Y,
-                                  reinterpret_cast<cudaStream_t>(stream), kWaitLimitNs, &e);
+    /* the block-scaled GEMM in its NVFP4 mode (tcgen05.mma kind::mxf4nvf4) */
+    int r = mx::launch_gemm(Xq, Xscale, M, K, Wq, Wscale, N, bias, Y, 4, nullptr,
+                            reinterpret_cast<cudaStream_t>(stream), kWaitLimitNs, &e, x_global_scale, w_global_scale);
     if (r == 1)
         return MXFP8_ERR_CUDA;
     return r == 0 ? MXFP8_OK : from_cuda(e);
@@ -463,8 +459,8 @@ mxfp8_status mxfp8_selftest_wait_timeout(int which, uint64_t timeout_ns, mxfp8_s
     switch (which) {
     case MXFP8_SELFTEST_GEMM:
         return from_cuda(mx::launch_wait_selftest(timeout_ns, s));
-    case MXFP8_SELFTEST_NVFP4_GEMM:
-        return from_cuda(mx::launch_nv_wait_selftest(timeout_ns, s));
+    case MXFP8_SELFTEST_NVFP4_GEMM: /* the same block-scaled GEMM kernel in its NVFP4 mode */
+        return from_cuda(mx::launch_wait_selftest(timeout_ns, s));
     case MXFP8_SELFTEST_ROWWISE_QUANT:
         return from_cuda(mx::launch_rw_wait_selftest(timeout_ns, s));
     default:
@@ -477,11 +473,10 @@ mxfp8_status mxfp8_device_status(mxfp8_stream_t stream)
     cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess)
         return MXFP8_ERR_CUDA;
-    unsigned int word = 0, rw_word = 0, nv_word = 0;
-    if (mx::read_and_clear_status(&word) != cudaSuccess || mx::read_and_clear_rw_status(&rw_word) != cudaSuccess ||
-        mx::read_and_clear_nv_status(&nv_word) != cudaSuccess)
+    unsigned int word = 0, rw_word = 0;
+    if (mx::read_and_clear_status(&word) != cudaSuccess || mx::read_and_clear_rw_status(&rw_word) != cudaSuccess)
         return MXFP8_ERR_CUDA;
-    return (word | rw_word | nv_word) ? MXFP8_ERR_TIMEOUT : MXFP8_OK;
+    return (word | rw_word) ? MXFP8_ERR_TIMEOUT : MXFP8_OK;
 }
 
 } // extern "C"

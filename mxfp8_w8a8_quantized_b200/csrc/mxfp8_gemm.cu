@@ -102,23 +102,29 @@ enum EpiMode : int {
     EPI_QUANT = 1,      /* MXFP8 codes + scales of BF16(acc + bias) for the next linear */
     EPI_QUANT_GELU = 2, /* MXFP8 codes + scales of BF16(GELU(BF16(acc + bias))) */
     EPI_ROWWISE = 3,    /* per-channel FP8: no block scales; Y = BF16(acc sx[m] sw[n] + bias) */
+    EPI_NVFP4 = 4,      /* NVFP4 operands (E2M1, UE4M3 per 16); Y = BF16(alpha acc + bias) */
 };
 
-template <bool PAIR>
+/* FP4: packed E2M1 operands -- a 128-byte stage row holds 256 elements,
+ * four MMAs of K = 64, each with its own scale atom per 128 rows. */
+template <bool PAIR, bool FP4 = false>
 struct Cfg {
-    static constexpr int STAGES = PAIR ? 6 : 4;
+    static constexpr int K_ATOMS = FP4 ? 4 : 1;             /* scale atoms per 128 rows per stage */
+    static constexpr int STAGES = FP4 ? (PAIR ? 5 : 3) : (PAIR ? 6 : 4);
     static constexpr int TILE_M = PAIR ? 256 : 128; /* output rows per tile */
     static constexpr int TILE_N = 256;
     static constexpr uint32_t A_ROWS = 128;                 /* A rows staged per CTA */
     static constexpr uint32_t B_ROWS = PAIR ? 128 : 256;    /* B rows staged per CTA */
     static constexpr uint32_t A_BYTES = A_ROWS * BK;
     static constexpr uint32_t B_BYTES = B_ROWS * BK;
-    static constexpr uint32_t SFA_BYTES = 512;              /* one atom: this CTA's 128 A rows */
-    static constexpr uint32_t SFB_BYTES = 1024;             /* two atoms: all 256 B rows */
+    static constexpr uint32_t SFA_BYTES = 512 * K_ATOMS;    /* this CTA's 128 A rows */
+    static constexpr uint32_t SFB_BYTES = 1024 * K_ATOMS;   /* all 256 B rows: [row half][atom] */
     static constexpr uint32_t STAGE_TX = (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) * (PAIR ? 2u : 1u);
-    static constexpr uint32_t SFA_COL = 256;                /* + 4 per stage */
-    static constexpr uint32_t SFB_COL = 256 + 4 * STAGES;   /* + 8 per stage */
-    static_assert(SFB_COL + 8 * STAGES <= TMEM_COLS, "TMEM budget");
+    static constexpr uint32_t SFA_STEP = 4 * K_ATOMS;       /* TMEM columns per stage */
+    static constexpr uint32_t SFB_STEP = 8 * K_ATOMS;
+    static constexpr uint32_t SFA_COL = 256;
+    static constexpr uint32_t SFB_COL = 256 + SFA_STEP * STAGES;
+    static_assert(SFB_COL + SFB_STEP * STAGES <= TMEM_COLS, "TMEM budget");
     static constexpr uint32_t OFF_A = 0;
     static constexpr uint32_t OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr uint32_t OFF_SFA = OFF_B + STAGES * B_BYTES;
@@ -144,7 +150,9 @@ struct GemmParams {
     uint8_t *S;           /* output scales, tensor-core layout of [M, N] (quantizing modes) */
     const float *sx;      /* [M] row scales (EPI_ROWWISE) */
     const float *sw;      /* [N] column scales (EPI_ROWWISE) */
-    int M, N, K;
+    const float *gx, *gw; /* the two tensors' FP32 global scales (EPI_NVFP4) */
+    int M, N;
+    int K;                /* operand row bytes: K elements of E4M3, K / 2 of packed E2M1 */
     int m_pad;            /* M rounded up to 128: rows that own scale bytes */
     int sf_kgroups;       /* N / 128: scale atoms per 128 output rows */
     int num_m, num_n;     /* output tiles */
@@ -202,11 +210,13 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, unsi
     }
 }
 
-/* Epilogue writing Y = BF16(acc + bias): bias + BF16 rounding, 32 columns at
- * a time, staged through a 64-byte-swizzled smem box and written by one TMA
- * store per warp -- scattered per-row global stores would occupy the L1 /
+/* Epilogue writing Y = BF16(acc + bias) (ALPHA: Y = BF16(fma(alpha, acc,
+ * bias)), the NVFP4 layer): bias + BF16 rounding, 32 columns at a time,
+ * staged through a 64-byte-swizzled smem box and written by one TMA store
+ * per warp -- scattered per-row global stores would occupy the L1 /
  * shared-memory data path that feeds the tensor core. */
-__device__ __forceinline__ void epilogue_bf16(const uint32_t (&acc)[128], const GemmParams &p,
+template <bool ALPHA>
+__device__ __forceinline__ void epilogue_bf16(const uint32_t (&acc)[128], const GemmParams &p, float alpha,
                                               const CUtensorMap *tmap_y, int row0, int col0, int lane,
                                               uint32_t buf, uint32_t rowbase, uint32_t swz)
 {
@@ -236,8 +246,13 @@ __device__ __forceinline__ void epilogue_bf16(const uint32_t (&acc)[128], const 
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int a = 32 * c + 8 * j8 + 2 * j;
-                __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(acc[a]) + b[2 * j],
-                                                         __uint_as_float(acc[a + 1]) + b[2 * j + 1]);
+                __nv_bfloat162 v;
+                if constexpr (ALPHA)
+                    v = __floats2bfloat162_rn(fmaf(alpha, __uint_as_float(acc[a]), b[2 * j]),
+                                              fmaf(alpha, __uint_as_float(acc[a + 1]), b[2 * j + 1]));
+                else
+                    v = __floats2bfloat162_rn(__uint_as_float(acc[a]) + b[2 * j],
+                                              __uint_as_float(acc[a + 1]) + b[2 * j + 1]);
                 o[j] = *reinterpret_cast<uint32_t *>(&v);
             }
             st_shared_v4(rowbase + ((((uint32_t)j8) ^ swz) << 4), o[0], o[1], o[2], o[3]);
@@ -422,8 +437,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                       const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                       const __grid_constant__ CUtensorMap tmap_y, const GemmParams p)
 {
-    using C = Cfg<PAIR>;
-    constexpr bool BS = EPI != EPI_ROWWISE; /* MXFP8 block scales (else per-channel FP8) */
+    constexpr bool FP4 = EPI == EPI_NVFP4;  /* packed E2M1 operands, UE4M3 scales per 16 */
+    using C = Cfg<PAIR, FP4>;
+    constexpr bool BS = EPI != EPI_ROWWISE; /* block scales (else per-channel FP8) */
     constexpr uint32_t STAGE_TX = BS ? C::STAGE_TX : (C::A_BYTES + C::B_BYTES) * (PAIR ? 2u : 1u);
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -482,7 +498,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_ptr;
 
-    const int KB = p.K / BK;
+    const int KB = (p.K + BK - 1) / BK; /* a partial last step reads zeros past K */
     const int num_tiles = p.num_m * p.num_n;
     const unsigned long long lim = p.timeout_ns;
 
@@ -522,15 +538,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         tma_load_2d_pair(dA, &tmap_a, kb * BK, rowA, lead);
                         tma_load_2d_pair(dB, &tmap_b, kb * BK, rowB, lead);
                         if constexpr (BS) {
-                            tma_load_3d_pair(dSA, &tmap_sfa, 0, kb, rbA, lead);
-                            tma_load_3d_pair(dSB, &tmap_sfb, 0, kb, rbB, lead);
+                            tma_load_3d_pair(dSA, &tmap_sfa, 0, kb * C::K_ATOMS, rbA, lead);
+                            tma_load_3d_pair(dSB, &tmap_sfb, 0, kb * C::K_ATOMS, rbB, lead);
                         }
                     } else {
                         tma_load_2d(dA, &tmap_a, kb * BK, rowA, full);
                         tma_load_2d(dB, &tmap_b, kb * BK, rowB, full);
                         if constexpr (BS) {
-                            tma_load_3d(dSA, &tmap_sfa, 0, kb, rbA, full);
-                            tma_load_3d(dSB, &tmap_sfb, 0, kb, rbB, full);
+                            tma_load_3d(dSA, &tmap_sfa, 0, kb * C::K_ATOMS, rbA, full);
+                            tma_load_3d(dSB, &tmap_sfb, 0, kb * C::K_ATOMS, rbB, full);
                         }
                     }
                 }
@@ -539,7 +555,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     } else if (warp == 1) {
         /* ------------------------------------------------ MMA issuer */
         if (lane == 0 && rank == 0) {
-            const uint32_t idesc = BS ? idesc_mxf8_e4m3(C::TILE_M, C::TILE_N) : idesc_f8_e4m3(C::TILE_M, C::TILE_N);
+            const uint32_t idesc = FP4  ? idesc_nvf4(C::TILE_M, C::TILE_N)
+                                   : BS ? idesc_mxf8_e4m3(C::TILE_M, C::TILE_N)
+                                        : idesc_f8_e4m3(C::TILE_M, C::TILE_N);
             uint32_t it = 0, tl = 0;
             bool ok = true, any = false;
             for (int t = tile0; ok && t < num_tiles; t += tstep, ++tl) {
@@ -558,8 +576,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t tsfa = tmem + C::SFA_COL + 4 * s;
-                    const uint32_t tsfb = tmem + C::SFB_COL + 8 * s;
+                    const uint32_t tsfa = tmem + C::SFA_COL + C::SFA_STEP * s;
+                    const uint32_t tsfb = tmem + C::SFB_COL + C::SFB_STEP * s;
                     const uint32_t sfa_s = sbase + C::OFF_SFA + s * C::SFA_BYTES;
                     const uint32_t sfb_s = sbase + C::OFF_SFB + s * C::SFB_BYTES;
                     const uint64_t adesc = desc_kmajor_sw128(sbase + C::OFF_A + s * C::A_BYTES);
@@ -587,18 +605,31 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         (void)sfa_s;
                         (void)sfb_s;
 #pragma unroll
-                        for (int k = 0; k < BK / 32; ++k)
-                            tc_mma_mxf8_pair(tacc, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k),
-                                             idesc_with_sf_id(idesc, (uint32_t)k), tsfa, tsfb, (kb | k) != 0);
+                        for (int k = 0; k < BK / 32; ++k) {
+                            if constexpr (FP4) /* K = 64: scale atom k of A, atoms k of both B halves */
+                                tc_mma_nvf4_pair(tacc, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc,
+                                                 tsfa + 4u * k, tsfb + 8u * k, (kb | k) != 0);
+                            else /* K = 32: byte k of every scale word */
+                                tc_mma_mxf8_pair(tacc, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k),
+                                                 idesc_with_sf_id(idesc, (uint32_t)k), tsfa, tsfb, (kb | k) != 0);
+                        }
                         tc_commit_pair(bar_empty + 8 * s, (uint16_t)0x3);
                     } else {
-                        tc_cp_32x128b_warpx4(tsfa, desc_sf_32x16(sfa_s));
-                        tc_cp_32x128b_warpx4(tsfb, desc_sf_32x16(sfb_s));
-                        tc_cp_32x128b_warpx4(tsfb + 4, desc_sf_32x16(sfb_s + 512u));
 #pragma unroll
-                        for (int k = 0; k < BK / 32; ++k)
-                            tc_mma_mxf8(tacc, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k),
-                                        idesc_with_sf_id(idesc, (uint32_t)k), tsfa, tsfb, (kb | k) != 0);
+                        for (int k = 0; k < C::K_ATOMS; ++k) {
+                            tc_cp_32x128b_warpx4(tsfa + 4u * k, desc_sf_32x16(sfa_s + 512u * k));
+                            tc_cp_32x128b_warpx4(tsfb + 8u * k, desc_sf_32x16(sfb_s + 512u * k));
+                            tc_cp_32x128b_warpx4(tsfb + 8u * k + 4u, desc_sf_32x16(sfb_s + 512u * (C::K_ATOMS + k)));
+                        }
+#pragma unroll
+                        for (int k = 0; k < BK / 32; ++k) {
+                            if constexpr (FP4)
+                                tc_mma_nvf4(tacc, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc,
+                                            tsfa + 4u * k, tsfb + 8u * k, (kb | k) != 0);
+                            else
+                                tc_mma_mxf8(tacc, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k),
+                                            idesc_with_sf_id(idesc, (uint32_t)k), tsfa, tsfb, (kb | k) != 0);
+                        }
                         tc_commit(bar_empty + 8 * s);
                     }
                     any = true;
@@ -642,13 +673,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t tsfa = tmem + C::SFA_COL + 4 * s;
-                    const uint32_t tsfb = tmem + C::SFB_COL + 8 * s;
+                    const uint32_t tsfa = tmem + C::SFA_COL + C::SFA_STEP * s;
+                    const uint32_t tsfb = tmem + C::SFB_COL + C::SFB_STEP * s;
                     const uint32_t sfa_s = sbase + C::OFF_SFA + s * C::SFA_BYTES;
                     const uint32_t sfb_s = sbase + C::OFF_SFB + s * C::SFB_BYTES;
-                    tc_cp_32x128b_warpx4_pair(tsfa, desc_sf_32x16(sfa_s));
-                    tc_cp_32x128b_warpx4_pair(tsfb, desc_sf_32x16(sfb_s));
-                    tc_cp_32x128b_warpx4_pair(tsfb + 4, desc_sf_32x16(sfb_s + 512u));
+                    /* atom k of A to 4 columns; atoms k of the two B row halves to 8 */
+#pragma unroll
+                    for (int k = 0; k < C::K_ATOMS; ++k) {
+                        tc_cp_32x128b_warpx4_pair(tsfa + 4u * k, desc_sf_32x16(sfa_s + 512u * k));
+                        tc_cp_32x128b_warpx4_pair(tsfb + 8u * k, desc_sf_32x16(sfb_s + 512u * k));
+                        tc_cp_32x128b_warpx4_pair(tsfb + 8u * k + 4u, desc_sf_32x16(sfb_s + 512u * (C::K_ATOMS + k)));
+                    }
                     tc_commit_pair(bar_sffull + 8 * s, (uint16_t)0x1);
                 }
                 if (!ok)
@@ -657,6 +692,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
     } else {
         /* ------------------------------------------------ epilogue */
+        /* NVFP4: alpha = 1 / (g_x g_w); the product of two binary32 values is
+         * exact in binary64, the quotient rounded once there, then to binary32 */
+        const float alpha = EPI == EPI_NVFP4 ? (float)(1.0 / ((double)__ldg(p.gx) * (double)__ldg(p.gw))) : 1.0f;
         const int q = warp & 3;            /* TMEM sub-partition this warp may read */
         const int h = (warp - 2) >> 2;     /* column half of the 256-wide tile */
         uint32_t tl = 0;
@@ -688,7 +726,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const uint32_t rowbase = buf + (uint32_t)lane * 64u;
             const uint32_t swz = ((uint32_t)lane >> 1) & 3u;
             if constexpr (EPI == EPI_BF16)
-                epilogue_bf16(acc, p, &tmap_y, row0, col0, lane, buf, rowbase, swz);
+                epilogue_bf16<false>(acc, p, 1.0f, &tmap_y, row0, col0, lane, buf, rowbase, swz);
+            else if constexpr (EPI == EPI_NVFP4)
+                epilogue_bf16<true>(acc, p, alpha, &tmap_y, row0, col0, lane, buf, rowbase, swz);
             else if constexpr (EPI == EPI_ROWWISE)
                 epilogue_rowwise(acc, p, &tmap_y, row0, col0, lane, buf, rowbase, swz);
             else
@@ -746,18 +786,21 @@ static bool make_operand_map(CUtensorMap *m, const void *base, int64_t rows, int
                      CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-/* Scale array in the tensor-core layout viewed as [row blocks][K/128][128 u32]
- * (one 512-byte atom per (row block, K step)); box = `atoms` consecutive row
- * blocks of one K step.  Row blocks past the end read as zero. */
-static bool make_scale_map(CUtensorMap *m, const void *base, int64_t rows, int64_t K, uint32_t atoms)
+/* Scale array in the tensor-core layout viewed as [row blocks][kg][128 u32]
+ * (one 512-byte atom per (row block, K group): kg = K / 128 groups of E8M0
+ * scales for MXFP8, K / 64 of UE4M3 scales for NVFP4); box = `katoms`
+ * consecutive K groups of `atoms` consecutive row blocks (shared-memory order
+ * [row block][K group][512 B]).  Atoms past the end read as zero. */
+static bool make_scale_map(CUtensorMap *m, const void *base, int64_t rows, int64_t kg, uint32_t katoms,
+                           uint32_t atoms)
 {
     PFN_encodeTiled enc = get_encode_fn();
     if (!enc)
         return false;
-    const int64_t kg = K / 128, rb = (rows + 127) / 128;
+    const int64_t rb = (rows + 127) / 128;
     cuuint64_t dims[3] = {128, (cuuint64_t)kg, (cuuint64_t)rb};
     cuuint64_t strides[2] = {512, (cuuint64_t)(kg * 512)};
-    cuuint32_t box[3] = {128, 1, atoms};
+    cuuint32_t box[3] = {128, katoms, atoms};
     cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void *>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -803,23 +846,30 @@ static DevInfo *dev_info()
 }
 
 template <bool PAIR, int EPI>
+constexpr uint32_t smem_bytes()
+{
+    return Cfg<PAIR, EPI == EPI_NVFP4>::SMEM_BYTES;
+}
+
+template <bool PAIR, int EPI>
 static cudaError_t ensure_attr(DevInfo *d)
 {
     if (d->attr[PAIR][EPI])
         return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(mxfp8_gemm_kernel<PAIR, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)Cfg<PAIR>::SMEM_BYTES);
+                                         (int)smem_bytes<PAIR, EPI>());
     if (e == cudaSuccess)
         d->attr[PAIR][EPI] = true;
     return e;
 }
 
-static void pair_config(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attr, unsigned grid, cudaStream_t stream)
+static void pair_config(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attr, unsigned grid, cudaStream_t stream,
+                        uint32_t smem)
 {
     cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(GEMM_THREADS);
-    cfg.dynamicSmemBytes = Cfg<true>::SMEM_BYTES;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
@@ -841,7 +891,7 @@ static void check_pairs(DevInfo *d)
     }
     cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attr[1];
-    pair_config(cfg, attr, 2 * (unsigned)d->sms, nullptr);
+    pair_config(cfg, attr, 2 * (unsigned)d->sms, nullptr, smem_bytes<true, EPI_BF16>());
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, mxfp8_gemm_kernel<true, EPI_BF16>, &cfg) == cudaSuccess)
         d->max_pair_clusters = n;
@@ -860,12 +910,12 @@ static cudaError_t launch_variant(DevInfo *d, const CUtensorMap &ma, const CUten
     cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attr[1];
     if (PAIR) {
-        pair_config(cfg, attr, (unsigned)grid, stream);
+        pair_config(cfg, attr, (unsigned)grid, stream, smem_bytes<PAIR, EPI>());
     } else {
         cfg = {};
         cfg.gridDim = dim3((unsigned)grid);
         cfg.blockDim = dim3(GEMM_THREADS);
-        cfg.dynamicSmemBytes = Cfg<PAIR>::SMEM_BYTES;
+        cfg.dynamicSmemBytes = smem_bytes<PAIR, EPI>();
         cfg.stream = stream;
     }
     return cudaLaunchKernelEx(&cfg, mxfp8_gemm_kernel<PAIR, EPI>, ma, mb, msa, msb, my, p);
@@ -883,6 +933,8 @@ static cudaError_t launch_mode(DevInfo *d, int epi, const CUtensorMap &ma, const
         return launch_variant<PAIR, EPI_QUANT_GELU>(d, ma, mb, msa, msb, my, p, grid, stream);
     case EPI_ROWWISE:
         return launch_variant<PAIR, EPI_ROWWISE>(d, ma, mb, msa, msb, my, p, grid, stream);
+    case EPI_NVFP4:
+        return launch_variant<PAIR, EPI_NVFP4>(d, ma, mb, msa, msb, my, p, grid, stream);
     default:
         return launch_variant<PAIR, EPI_BF16>(d, ma, mb, msa, msb, my, p, grid, stream);
     }
@@ -903,14 +955,19 @@ static bool pair_enabled()
  * epi = 0: Y is BF16 [M, N], S unused.  epi = 1 / 2: Y receives E4M3 codes
  * [M, N] and S the tensor-core scales of [M, N] (2: GELU before the
  * quantization); N % 128 == 0.  epi = 3 (per-channel FP8): Xs / Ws are FP32
- * row scales [M] / [N], Y is BF16 [M, N].
+ * row scales [M] / [N], Y is BF16 [M, N].  epi = 4 (NVFP4): Xq / Wq are packed
+ * E2M1 codes [M, K/2] / [N, K/2], Xs / Ws their UE4M3 scales in the
+ * tensor-core layout of 16-element blocks, gx / gw the device global scales,
+ * Y is BF16 [M, N]; K % 64 == 0.
  * Returns 0 ok, 1 tensor-map failure, 2 CUDA error (in *err).
  */
 int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void *Wq, const void *Ws, int64_t N,
                 const void *bias, void *Y, int epi, void *S, cudaStream_t stream, unsigned long long timeout_ns,
-                cudaError_t *err)
+                cudaError_t *err, const float *gx, const float *gw)
 {
     const bool bs = epi != EPI_ROWWISE;
+    const bool fp4 = epi == EPI_NVFP4;
+    const int64_t kbytes = fp4 ? K / 2 : K; /* operand row bytes */
     *err = cudaSuccess;
     if (M == 0)
         return 0;
@@ -928,12 +985,16 @@ int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void
 
     const uint32_t b_rows = pair ? Cfg<true>::B_ROWS : Cfg<false>::B_ROWS;
     CUtensorMap ma, mb, msa, msb, my;
-    const bool out_ok = (epi == EPI_BF16 || epi == EPI_ROWWISE) ? make_output_map(&my, Y, M, N)
-                                                                 : make_codes_out_map(&my, Y, M, N);
-    if (!make_operand_map(&ma, Xq, M, K, 128) || !make_operand_map(&mb, Wq, N, K, b_rows) || !out_ok)
+    const bool out_ok = (epi == EPI_BF16 || epi == EPI_ROWWISE || fp4) ? make_output_map(&my, Y, M, N)
+                                                                         : make_codes_out_map(&my, Y, M, N);
+    if (!make_operand_map(&ma, Xq, M, kbytes, 128) || !make_operand_map(&mb, Wq, N, kbytes, b_rows) || !out_ok)
         return 1;
     if (bs) {
-        if (!make_scale_map(&msa, Xs, M, K, 1) || !make_scale_map(&msb, Ws, N, K, 2))
+        /* K groups of scale atoms: 128 elements (E8M0) or 64 (UE4M3); the
+         * GEMM takes one group per 128-byte step, or four */
+        const int64_t kg = fp4 ? (K + 63) / 64 : K / 128;
+        const uint32_t katoms = fp4 ? 4u : 1u;
+        if (!make_scale_map(&msa, Xs, M, kg, katoms, 1) || !make_scale_map(&msb, Ws, N, kg, katoms, 2))
             return 1;
     } else {
         msa = ma; /* not read without block scales */
@@ -945,19 +1006,22 @@ int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void
     p.S = static_cast<uint8_t *>(S);
     p.sx = bs ? nullptr : static_cast<const float *>(Xs);
     p.sw = bs ? nullptr : static_cast<const float *>(Ws);
+    p.gx = gx;
+    p.gw = gw;
     p.M = (int)M;
     p.N = (int)N;
-    p.K = (int)K;
+    p.K = (int)kbytes;
     p.m_pad = (int)((M + 127) / 128 * 128);
     p.sf_kgroups = (int)(N / 128);
     const int tile_m = pair ? Cfg<true>::TILE_M : Cfg<false>::TILE_M;
     p.num_m = (int)((M + tile_m - 1) / tile_m);
     p.num_n = (int)((N + 255) / 256);
-    const int64_t n_group = std::min<int64_t>(p.num_n, RASTER_B_GROUP_BYTES / ((int64_t)Cfg<true>::TILE_N * K));
+    const int64_t n_group =
+        std::min<int64_t>(p.num_n, RASTER_B_GROUP_BYTES / ((int64_t)Cfg<true>::TILE_N * kbytes));
     if (n_group >= RASTER_MIN_N_GROUP)
         p.raster = -(int)n_group;
     else
-        p.raster = (int64_t)N * K > RASTER_LARGE_B_BYTES ? RASTER_LARGE_B : RASTER_SMALL_B;
+        p.raster = (int64_t)N * kbytes > RASTER_LARGE_B_BYTES ? RASTER_LARGE_B : RASTER_SMALL_B;
     p.timeout_ns = timeout_ns;
     const int tiles = p.num_m * p.num_n;
     cudaError_t e;

@@ -293,6 +293,30 @@ __device__ __forceinline__ void tc_mma_mxf8_pair(uint32_t tacc, uint64_t adesc, 
         : "memory");
 }
 
+/* D(tmem) (+)= A(smem) . B(smem)^T with packed E2M1 operands and UE4M3
+ * scales per 16 elements (K = 64 per instruction: 32 bytes of each operand
+ * row; each row's four scale bytes of the step fill one 32-bit TMEM word). */
+__device__ __forceinline__ void tc_mma_nvf4(uint32_t tacc, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t tsfa, uint32_t tsfb, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p;\n\t}\n" ::"r"(tacc),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(tsfa), "r"(tsfb), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_nvf4_pair(uint32_t tacc, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t tsfa, uint32_t tsfb, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p;\n\t}\n" ::"r"(tacc),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(tsfa), "r"(tsfb), "r"(accumulate)
+        : "memory");
+}
+
 /* D(tmem) (+)= A(smem) . B(smem)^T, E4M3 x E4M3 without block scales, 32-wide
  * K, over the CTA pair (same operand split as tc_mma_mxf8_pair). */
 __device__ __forceinline__ void tc_mma_f8_pair(uint32_t tacc, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -363,6 +387,17 @@ __host__ __device__ constexpr uint32_t idesc_mxf8_e4m3(int M, int N)
 __host__ __device__ constexpr uint32_t idesc_f8_e4m3(int M, int N)
 {
     return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+/*
+ * Instruction descriptor of kind::mxf4nvf4 with 16-element blocks: A and B
+ * E2M1 (1 at [7,10) and [10,13)), both K-major, N >> 3 at [17,23), scale
+ * type UE4M3 (0 at bit 23), M >> 4 at [24,29), dense K = 64 (0 at bit 31).
+ * An instruction uses all four scale bytes of its TMEM word (scale-factor
+ * IDs 0).
+ */
+__host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N)
+{
+    return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (0u << 23) | ((uint32_t)(M >> 4) << 24);
 }
 __host__ __device__ constexpr uint32_t idesc_with_sf_id(uint32_t idesc, uint32_t id)
 {

@@ -147,7 +147,8 @@ def test_nvfp4_accounting():
     assert wl.flops() == 2.0 * M * N * K
     assert wl.quant_bytes() == M * K * 2 + M * K // 2 + M * K // 16
     assert wl.gemm_bytes() == pytest.approx((M + N) * K * 9 / 16 + 2 * M * N + 2 * N)
-    assert wl.tc_over_bf16 == 1.0 and wl.profile_kernel == "nvfp4_gemm"
+    # the 4-bit block-scaled kind: the FP4 peak is the BF16 figure x 4
+    assert wl.tc_over_bf16 == bench.FP4_OVER_BF16 == 4.0 and wl.profile_kernel == "mxfp8_gemm"
     with pytest.raises(ValueError):
         bench.make_workload("c2_ffn_pair_832x1104", scheme="nvfp4")
 
@@ -161,16 +162,16 @@ def test_traffic_is_reported_only_for_the_profiled_kernel_files(tmp_path, monkey
     prof = tmp_path / "profiles"
     prof.mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    for kernel in ("mxfp8_gemm", "nvfp4_gemm"):
-        (prof / f"{kernel}_k.json").write_text(json.dumps(
-            {"kernel_source_sha": build.source_sha(kernel), "dram_bytes_per_launch": 123}))
-        assert bench.load_traffic("k", kernel) == 123
-        (prof / f"{kernel}_k.json").write_text(json.dumps(
-            {"kernel_source_sha": "0" * 16, "dram_bytes_per_launch": 123}))
-        assert bench.load_traffic("k", kernel) is None
+    kernel = "mxfp8_gemm"
+    (prof / f"{kernel}_k.json").write_text(json.dumps(
+        {"kernel_source_sha": build.source_sha(kernel), "dram_bytes_per_launch": 123}))
+    assert bench.load_traffic("k", kernel) == 123
+    (prof / f"{kernel}_k.json").write_text(json.dumps(
+        {"kernel_source_sha": "0" * 16, "dram_bytes_per_launch": 123}))
+    assert bench.load_traffic("k", kernel) is None
     assert bench.load_traffic("missing", "mxfp8_gemm") is None
-    # the two kernels hash different file sets; the library hash covers both
-    assert build.source_sha("mxfp8_gemm") != build.source_sha("nvfp4_gemm") != build.source_sha()
+    # the GEMM's hash covers its own files only; the library hash covers all
+    assert build.source_sha("mxfp8_gemm") != build.source_sha()
 
 
 def test_reference_arm_times_the_whole_chain():

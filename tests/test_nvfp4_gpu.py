@@ -2,8 +2,9 @@
 and UE4M3 scales bit-exact (both sides take the same binary32 steps), the
 tensor amax and the global scale exact -- the GPU forms its global scale on
 the device, the oracle forms its own from the host copy of the same tensor,
-and the two must be the same binary32 value -- and the GEMM within the
-output tolerance."""
+and the two must be the same binary32 value -- and the GEMM (the block-scaled
+GEMM in its 4-bit mode, on CTA pairs and, in a child process, on single
+CTAs) within the output tolerance."""
 import numpy as np
 import pytest
 import torch
@@ -193,3 +194,17 @@ def test_gemm_argument_errors(mx):
         mx.nvfp4_gemm(xq, xs, wq, ws, 1.0, one)
     with pytest.raises(ValueError):
         mx.nvfp4_quantize(x, torch.ones(2, device="cuda"))
+
+
+def test_gemm_single_cta_variant_in_subprocess():
+    # the GEMM has a CTA-pair (default) and a single-CTA variant, fixed per
+    # process; the NVFP4 GEMM checks run again in a child on single CTAs
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    env = dict(os.environ, MXFP8_GEMM_PAIR="0")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider", "-m", "gpu",
+                        os.path.join(here, "test_nvfp4_gpu.py"), "-k", "gemm and not subprocess"],
+                       env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
