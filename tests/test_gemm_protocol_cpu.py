@@ -1,5 +1,5 @@
-"""CPU model of the block-scaled MXFP8 GEMM's barrier protocol on CTA pairs
-(no GPU).
+"""CPU model of the block-scaled GEMM's barrier protocol on CTA pairs (no
+GPU).
 
 The kernel's roles, reduced to their mbarrier traffic:
   * per CTA, a TMA producer filling a ring of STAGES stages -- the A and B
@@ -24,13 +24,13 @@ Random interleavings must finish without a copy reading scales of another
 K step, a TMEM scale column being overwritten before the MMAs that read it
 ran, the MMA reading an operand stage or scale column that holds another K
 step, a stage being reloaded while it is read, or the accumulator being
-reused before it is drained; planted protocol mistakes must be caught.
+reused before it is drained; planted protocol mistakes must be caught.  The
+ring depth is that of the E4M3 mode (6 stages) and of the NVFP4 mode (5
+stages, the same barriers with four times the scale copies per stage).
 """
 import random
 
 import pytest
-
-STAGES = 6
 
 
 class Bar:
@@ -51,7 +51,7 @@ class Deadlock(Exception):
     pass
 
 
-def run(num_tiles, KB, seed, mutation=None):
+def run(num_tiles, KB, seed, mutation=None, STAGES=6):
     rnd = random.Random(seed)
     bars = {}
     for cta in range(2):
@@ -198,11 +198,12 @@ def run(num_tiles, KB, seed, mutation=None):
         last, live = state, nxt
 
 
+@pytest.mark.parametrize("stages", [6, 5])
 @pytest.mark.parametrize("KB", [1, 2, 5, 7, 11, 40])
 @pytest.mark.parametrize("tiles", [1, 2, 3, 5])
-def test_protocol_completes_and_hands_off_the_right_buffers(KB, tiles):
+def test_protocol_completes_and_hands_off_the_right_buffers(KB, tiles, stages):
     for seed in range(3):
-        run(tiles, KB, seed)
+        run(tiles, KB, seed, STAGES=stages)
 
 
 @pytest.mark.parametrize("mutation,KB,tiles", [
