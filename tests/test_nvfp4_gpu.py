@@ -133,6 +133,27 @@ def test_gemm_within_tolerance(mx, M, K, N):
     assert_within_tol(bf16_values(bf16_bits(y)), yref, f"nvfp4 {M}x{K}x{N}")
 
 
+# The tile walk is chosen on the packed row bytes (K / 2): one shape per
+# walk, each with several groups, a reversed group and a ragged last group,
+# sampled in every 128 x 128 quarter of every 256 x 256 tile.
+@pytest.mark.parametrize("M,K,N", [
+    (300, 40960, 4864),    # N-tile groups of 9: 9 + 9 + 1 of 19 N tiles
+    (2600, 512, 1024),     # M-tile groups of 8: 8 + 3 of 11 M tiles
+    (4400, 65536, 2048),   # M-tile groups of 16 (packed weights 67 MB): 16 + 2 of 18 M tiles
+])
+def test_gemm_tile_walk_covers_every_tile(mx, M, K, N):
+    x, w, b, (gx, gx_ref), (gw, gw_ref), wq, ws = _nv_layer(mx, M, K, N, seed=M + N)
+    xq, xs = mx.nvfp4_quantize(x, gx)
+    y = mx.nvfp4_gemm(xq, xs, wq, ws, gx, gw, b)
+    torch.cuda.synchronize()
+    assert mx.device_status() == 0
+    rows = sorted({min(r, M - 1) for t in range(0, M, 128) for r in (t, t + 77, t + 127)})
+    cols = sorted({min(c, N - 1) for t in range(0, N, 128) for c in (t, t + 50, t + 127)})
+    yref = _oracle_y(x, w, b, gx_ref, gw_ref, rows=np.array(rows), cols=np.array(cols))
+    got = bf16_values(bf16_bits(y))[np.ix_(rows, cols)]
+    assert_within_tol(got, yref, f"nvfp4 tile walk {M}x{K}x{N}")
+
+
 def test_gemm_exact_grid_values(mx):
     # every block holds a 6 and values of the E2M1 grid; with g = 1 every
     # scale is exactly 1 (6 * RN(1/6) rounds to 1 in E4M3), the codes are
