@@ -78,15 +78,21 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0; /* 256 FP32 columns */
 /* Tile walk (tile_coords).  Preferred: groups of N tiles whose weight rows
  * (at most RASTER_B_GROUP_BYTES) stay in L2 while the activation rows
- * stream past them once per group -- used when such a group spans at least
- * RASTER_MIN_N_GROUP N tiles.  Measured DRAM reads per launch at M = 75348
- * (81 frames at 832x1104): N = K = 5120 705 -> 473 MB (the whole weight
- * resident, A read once), ffn.net.0.proj 1.93 -> 1.58 GB.  Otherwise (long K:
- * a weight tile is too large for a useful group) groups of M tiles walk every
- * N tile: 8 when the weights fit in L2 alongside them, 16 when they are
- * re-read from DRAM once per group. */
-constexpr int64_t RASTER_B_GROUP_BYTES = 48ll << 20;
-constexpr int RASTER_MIN_N_GROUP = 8;
+ * stream past them once per group -- used when such a group can span at
+ * least RASTER_MIN_N_GROUP N tiles; the N tiles are split into the fewest
+ * groups of that size, made equal (60 tiles: 20 + 20 + 20, not 24 + 24 + 12).
+ * DRAM reads per launch at M = 75348 (81 frames at 832x1104), ncu, cold L2,
+ * by N tiles per group:
+ *   q/k/v (K 5120, N 15360)          38: 3.40 GB, 24: 2.87, 18: 3.36, all 60: 8.08
+ *   ffn.net.0.proj (K 5120, N 13824)  38: 3.36 GB, 27: 2.23, 18: 2.19, all 54: 7.21
+ *   ffn.net.2 (K 13824, N 5120)       13: 8.04 GB, 10: 7.26, 7: 7.67, all 20: 9.33
+ * (groups of more weight are re-read from DRAM on every wave of tiles; this
+ * rule takes 20, 27 and 10).  Otherwise (long K: a weight tile is too large
+ * for a useful group) groups of M tiles walk every N tile: 8 when the
+ * weights fit in L2 alongside them, 16 when they are re-read from DRAM once
+ * per group. */
+constexpr int64_t RASTER_B_GROUP_BYTES = 36ll << 20;
+constexpr int RASTER_MIN_N_GROUP = 6;
 constexpr int RASTER_SMALL_B = 8, RASTER_LARGE_B = 16;
 constexpr int64_t RASTER_LARGE_B_BYTES = 48ll << 20;
 /* mbarrier.try_wait suspend-time hints (ns): the producer and MMA threads wait
@@ -1016,11 +1022,12 @@ int launch_gemm(const void *Xq, const void *Xs, int64_t M, int64_t K, const void
     const int tile_m = pair ? Cfg<true>::TILE_M : Cfg<false>::TILE_M;
     p.num_m = (int)((M + tile_m - 1) / tile_m);
     p.num_n = (int)((N + 255) / 256);
-    const int64_t n_group =
+    const int64_t n_fit =
         std::min<int64_t>(p.num_n, RASTER_B_GROUP_BYTES / ((int64_t)Cfg<true>::TILE_N * kbytes));
-    if (n_group >= RASTER_MIN_N_GROUP)
-        p.raster = -(int)n_group;
-    else
+    if (n_fit >= RASTER_MIN_N_GROUP) {
+        const int64_t groups = (p.num_n + n_fit - 1) / n_fit;
+        p.raster = -(int)((p.num_n + groups - 1) / groups);
+    } else
         p.raster = (int64_t)N * kbytes > RASTER_LARGE_B_BYTES ? RASTER_LARGE_B : RASTER_SMALL_B;
     p.timeout_ns = timeout_ns;
     const int tiles = p.num_m * p.num_n;

@@ -59,14 +59,15 @@ def test_linear_vs_oracle(mx, M, K, N):
     assert np.isfinite(y).all()
 
 
-# One shape per tile walk of the GEMM (groups of N tiles holding up to 48 MB
-# of weight rows when such a group spans at least 8 N tiles; else groups of
-# 8 M tiles, or 16 when the weights exceed 48 MB), each with several groups,
-# an odd group (walked in reverse) and a ragged last group.  Rows and columns
+# One shape per tile walk of the GEMM (equal groups of N tiles, each holding
+# at most 36 MB of weight rows, when a group of that size spans at least 6 N
+# tiles; else groups of 8 M tiles, or 16 when the weights exceed 48 MB), each
+# with several groups, an odd group (walked in reverse) and a ragged last
+# group.  Rows and columns
 # are sampled in every 128 x 128 quarter of every 256 x 256 tile, so a tile
 # the walk skipped or visited twice shows.
 @pytest.mark.parametrize("M,K,N", [
-    (300, 20480, 4864),    # N-tile groups of 9: 9 + 9 + 1 of 19 N tiles, two M tiles (ragged)
+    (300, 20480, 4864),    # N-tile groups of 7: 7 + 7 + 5 of 19 N tiles, two M tiles (ragged)
     (2600, 256, 1024),     # M-tile groups of 8: 8 + 3 of 11 M tiles, four N tiles
     (4400, 32768, 2048),   # M-tile groups of 16 (weights 67 MB): 16 + 2 of 18 M tiles
 ])
